@@ -1,0 +1,212 @@
+/*
+ * flce.h - C ABI of the B200 (sm_100a) fused linear cross-entropy library.
+ *
+ * The operation. "Liger Kernel: Efficient Triton Kernels for LLM Training"
+ * (paper review, 提案手法; Figure 1 "Fused Linear Cross Entropy") describes a
+ * chunked fusion of the lm_head projection with cross-entropy that never keeps
+ * the logits over the whole vocabulary. "Liger-Kernel 項目詳細介紹"
+ * (使用方法 > 3. 低級 API 方式) gives its call, loss_fn(weight, input, target),
+ * with weight [V,H], input [BT,H] and an integer target [BT], and says under
+ * 核心特性 > 技術實現 that nothing is approximated. So, exactly:
+ *
+ *     z = X W^T;  l_i = logsumexp(z_i) - z_{i,t_i} for rows with t_i != ignore_index;
+ *     loss = sum_i l_i / N (FLCE_MEAN, N = non-ignored rows) or sum_i l_i (FLCE_SUM);
+ *     dz_i = (softmax(z_i) - onehot(t_i)) * (1/N or 1), 0 for ignored rows;
+ *     grad_X = dz W;  grad_W = dz^T X.
+ *
+ * The gradients are those of the loss for an upstream gradient of 1. N = 0
+ * (every row ignored) gives loss 0 and zero gradients.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers in flce_tensor are DEVICE pointers on the current CUDA device.
+ *    The caller owns every tensor; the library never keeps a pointer after a
+ *    call returns (work it enqueued still reads them until it completes).
+ *  - Matrices are row-major: stride[1] == 1, stride[0] >= shape[1] (elements).
+ *  - Work is enqueued on `stream` (a cudaStream_t / CUstream; NULL = legacy
+ *    default stream). Nothing synchronises unless FLCE_FLAG_SYNC_CHECK is set.
+ *  - A call returns FLCE_OK once its work is enqueued. Argument errors are
+ *    found on the host before anything is enqueued and leave outputs untouched.
+ *    Data errors found on the device (a target outside [0,V) that is not
+ *    ignore_index) set a bit of the device error word, read with
+ *    flce_get_device_error(); such rows are treated as ignored. Nothing traps.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef FLCE_H
+#define FLCE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLCE_VERSION 100 /* 1.0.0 */
+
+#if defined(__GNUC__)
+#define FLCE_API __attribute__((visibility("default")))
+#else
+#define FLCE_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* flce_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  FLCE_OK = 0,
+  FLCE_ERR_INVALID_ARG = 1,        /* null pointer, bad shape, stride or alignment */
+  FLCE_ERR_UNSUPPORTED_DTYPE = 2,  /* dtype combination not provided */
+  FLCE_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 (B200); caller may fall back */
+  FLCE_ERR_ALLOC = 4,              /* stream-ordered workspace allocation failed */
+  FLCE_ERR_CUDA = 5,               /* a CUDA runtime call failed */
+  FLCE_ERR_WORKSPACE_TOO_SMALL = 6 /* caller-provided workspace smaller than the plan needs */
+} flce_status;
+
+typedef enum { FLCE_F32 = 0, FLCE_BF16 = 1, FLCE_I64 = 2 } flce_dtype;
+typedef enum { FLCE_MEAN = 0, FLCE_SUM = 1 } flce_reduction;
+
+/* Bits of the device error word. */
+#define FLCE_DEVERR_TARGET_RANGE 0x1u /* a target outside [0,V) that is not ignore_index */
+#define FLCE_DEVERR_TIMEOUT 0x2u      /* a bounded wait inside a kernel ran out; results invalid */
+
+/* A dense tensor of rank 0, 1 or 2. */
+typedef struct {
+  void* data;        /* device pointer */
+  int32_t dtype;     /* flce_dtype */
+  int32_t ndim;      /* 0, 1 or 2 */
+  int64_t shape[2];  /* shape[0..ndim-1] */
+  int64_t stride[2]; /* in elements; the last stride must be 1 */
+} flce_tensor;
+
+/* How grad_W is accumulated across row chunks. */
+typedef enum {
+  FLCE_GRADW_ACCUM_OUTPUT = 0, /* fp32 sum per chunk, added into grad_W in its own dtype */
+  FLCE_GRADW_ACCUM_FP32 = 1    /* fp32 V x H accumulator in the workspace, cast once */
+} flce_gradw_accum;
+
+#define FLCE_FLAG_SYNC_CHECK 0x1  /* synchronise and check for CUDA errors after each launch */
+#define FLCE_FLAG_TIME_PHASES 0x2 /* record CUDA events around each phase (flce_phase_times) */
+
+typedef struct {
+  int64_t chunk_rows;            /* rows per chunk; 0 = chosen from workspace_limit_bytes.
+                                    Rounded up to a multiple of 128. */
+  int64_t workspace_limit_bytes; /* chunk store budget; 0 = at most 512 MiB and at most half
+                                    the rows, so two or more chunks whenever BT > 128 */
+  void* workspace;               /* optional caller-owned device workspace (256-byte aligned) */
+  int64_t workspace_bytes;       /* its size in bytes */
+  int32_t grad_w_accum;          /* flce_gradw_accum */
+  int32_t flags;                 /* FLCE_FLAG_* */
+  const int64_t* n_valid;        /* optional DEVICE pointer: the mean denominator N to use
+                                    (e.g. the count over all data-parallel ranks, from
+                                    flce_count_valid + an all-reduce). NULL = count locally. */
+  float* row_loss;               /* optional DEVICE [BT] fp32: per-row losses l_i (0 if ignored) */
+  float* lse;                    /* optional DEVICE [BT] fp32: per-row logsumexp of z_i */
+} flce_options;
+
+typedef struct {
+  int64_t chunk_rows;                /* rows per chunk actually used */
+  int64_t n_chunks;                  /* number of chunks */
+  int64_t workspace_bytes;           /* peak extra device memory this call uses */
+  int64_t materialized_logits_bytes; /* BT * V * 2: the logits a non-fused loss would hold */
+  int32_t kernel_launches;           /* kernels this call enqueued */
+  int32_t path;                      /* 0 = SIMT fp32 path, 1 = tcgen05 bf16 path */
+} flce_stats;
+
+/* Fill *opt with the defaults (all zero / NULL). */
+FLCE_API void flce_options_init(flce_options* opt);
+
+/*
+ * Fused linear cross-entropy, forward and backward, in one call.
+ *   X       [BT,H]  bf16 or f32 (row-major)
+ *   W       [V,H]   same dtype as X
+ *   target  [BT]    int64; rows equal to ignore_index are ignored
+ *   reduction       FLCE_MEAN or FLCE_SUM
+ *   loss    scalar  f32 (ndim 0, or ndim 1 with one element): written
+ *   grad_X  [BT,H]  same dtype as X, or NULL to skip: fully overwritten
+ *   grad_W  [V,H]   same dtype as W, or NULL to skip: fully overwritten
+ * bf16 runs the tcgen05 tensor-core path (fp32 accumulation, bf16 results,
+ * H % 8 == 0, 16-byte aligned rows); f32 runs an exact-fp32 SIMT path.
+ * Workspace is taken stream-ordered (cudaMallocAsync) and released at the end.
+ */
+FLCE_API flce_status flce_fwd_bwd(const flce_tensor* X, const flce_tensor* W, const flce_tensor* target,
+                         int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                         flce_tensor* grad_X, flce_tensor* grad_W, flce_stream_t stream);
+
+/* As flce_fwd_bwd, with options (opt may be NULL) and statistics (stats may be NULL). */
+FLCE_API flce_status flce_fwd_bwd_ex(const flce_tensor* X, const flce_tensor* W,
+                            const flce_tensor* target, int64_t ignore_index, int32_t reduction,
+                            flce_tensor* loss, flce_tensor* grad_X, flce_tensor* grad_W,
+                            flce_stream_t stream, const flce_options* opt, flce_stats* stats);
+
+/*
+ * Host-only planning: fills *out with the chunk rows, chunk count and
+ * workspace bytes flce_fwd_bwd_ex would use for this shape. Touches no GPU.
+ * dtype is FLCE_BF16 or FLCE_F32. want_grad_W selects whether a grad_W
+ * accumulator (FLCE_GRADW_ACCUM_FP32) is counted.
+ */
+FLCE_API flce_status flce_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, int32_t want_grad_W,
+                      const flce_options* opt, flce_stats* out);
+
+/*
+ * N, the count of rows whose target is not ignore_index, written as int64
+ * to the DEVICE pointer n_valid_out on `stream`. Targets outside [0,V) that
+ * are not ignore_index set FLCE_DEVERR_TARGET_RANGE and are not counted.
+ * Used by data-parallel callers to all-reduce N before flce_fwd_bwd_ex.
+ */
+FLCE_API flce_status flce_count_valid(const flce_tensor* target, int64_t V, int64_t ignore_index,
+                             int64_t* n_valid_out, flce_stream_t stream);
+
+/*
+ * Cross-entropy of given logits (the logits-given CrossEntropy of the paper
+ * review's 主な発見: online softmax with in-place gradient replacement).
+ *   logits [BT,V] bf16 or f32; target [BT] int64; loss scalar f32.
+ *   grad_logits: same shape/dtype as logits, or NULL to skip. It may be the
+ *   logits tensor itself (in-place gradient replacement).
+ * opt may be NULL; only opt->n_valid, opt->row_loss and opt->lse are read.
+ */
+FLCE_API flce_status flce_cross_entropy(const flce_tensor* logits, const flce_tensor* target,
+                               int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                               flce_tensor* grad_logits, flce_stream_t stream,
+                               const flce_options* opt);
+
+/*
+ * Plain bf16 GEMM on the library's tcgen05 engine, for testing that engine
+ * on its own: C[M,N] (f32, row-major, ldc) = sum_k A(m,k) * B(n,k).
+ * A is [M,K] row-major (a_mn_major = 0, lda >= K) or [K,M] row-major
+ * (a_mn_major = 1, lda >= M); B likewise with N. Leading dimensions are in
+ * elements and must be multiples of 8; pointers 16-byte aligned.
+ */
+FLCE_API flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N,
+                           int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn_major,
+                           int32_t b_mn_major, flce_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns the device error word of the current
+ * device in *err (FLCE_DEVERR_* bits) and clears it. The word is shared by
+ * every stream on the device.
+ */
+FLCE_API flce_status flce_get_device_error(flce_stream_t stream, uint32_t* err);
+
+/*
+ * Phase timing (calls made with FLCE_FLAG_TIME_PHASES): waits for the
+ * recorded events and writes, for each phase p < n_phases, the summed
+ * milliseconds to ms[p] and the number of timed launches to count[p] (either
+ * may be NULL). reset != 0 clears the record afterwards. Phases:
+ *   0 count valid rows, 1 logits GEMM + online-softmax epilogue,
+ *   2 row combine + loss, 3 in-place dlogits, 4 grad_X / grad_W GEMMs,
+ *   5 final loss reduction.
+ */
+#define FLCE_NUM_PHASES 6
+FLCE_API flce_status flce_phase_times(double* ms, int32_t* count, int32_t n_phases, int32_t reset);
+
+/* Static string for a status code. */
+FLCE_API const char* flce_status_string(int32_t status);
+
+/* FLCE_VERSION of the built library. */
+FLCE_API int32_t flce_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLCE_H */

@@ -1,0 +1,193 @@
+"""Public Python API over the C ABI (argument marshalling only).
+
+fused_linear_cross_entropy(X, W, target) runs the whole path (loss, grad_X,
+grad_W) in the CUDA library in one call. FusedLinearCrossEntropyLoss mirrors
+the low-level API of "Liger-Kernel 項目詳細介紹" (使用方法 > 3. 低級 API 方式):
+loss_fn(lm_head.weight, input, target) followed by loss.backward().
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _binding as B
+
+_RED = {"mean": B.MEAN, "sum": B.SUM}
+_ACC = {"output": B.GRADW_ACCUM_OUTPUT, "fp32": B.GRADW_ACCUM_FP32}
+
+
+def _options(chunk_rows=0, workspace_limit_bytes=0, grad_w_accum="output", flags=0,
+             n_valid=None, row_loss=None, lse=None, workspace=None):
+    o = B.FlceOptions()
+    B.lib().flce_options_init(ctypes.byref(o))
+    o.chunk_rows = int(chunk_rows)
+    o.workspace_limit_bytes = int(workspace_limit_bytes)
+    o.grad_w_accum = _ACC[grad_w_accum]
+    o.flags = int(flags)
+    o.n_valid = None if n_valid is None else n_valid.data_ptr()
+    o.row_loss = None if row_loss is None else row_loss.data_ptr()
+    o.lse = None if lse is None else lse.data_ptr()
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    return o
+
+
+def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor,
+                               ignore_index: int = -100, reduction: str = "mean",
+                               want_grad_X: bool = True, want_grad_W: bool = True,
+                               chunk_rows: int = 0, workspace_limit_bytes: int = 0,
+                               grad_w_accum: str = "output", n_valid: Optional[torch.Tensor] = None,
+                               row_loss: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                               flags: int = 0, stream=None, out=None, return_stats: bool = False):
+    """Loss, grad_X and grad_W of cross-entropy over X W^T in one call.
+
+    X [BT, H] and W [V, H] (bf16 or fp32, CUDA), target [BT] int64.
+    Tensors on the host are staged to the current CUDA device and the
+    results copied back (the end-to-end path); nothing runs on the CPU.
+    out = (loss, grad_X, grad_W) preallocated device tensors may be given.
+    Returns (loss [scalar fp32], grad_X or None, grad_W or None[, stats]).
+    """
+    host = not X.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        X = X.to(dev, non_blocking=True)
+        W = W.to(dev, non_blocking=True)
+        target = target.to(dev, non_blocking=True)
+    if out is not None:
+        loss, gX, gW = out
+    else:
+        loss = torch.empty((), dtype=torch.float32, device=X.device)
+        gX = torch.empty_like(X) if want_grad_X else None
+        gW = torch.empty_like(W) if want_grad_W else None
+    o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags, n_valid, row_loss, lse)
+    st = B.FlceStats()
+    tX, tW, tt, tl = B.tensor(X), B.tensor(W), B.tensor(target), B.tensor(loss)
+    tgX = B.tensor(gX) if gX is not None else None
+    tgW = B.tensor(gW) if gW is not None else None
+    rc = B.lib().flce_fwd_bwd_ex(ctypes.byref(tX), ctypes.byref(tW), ctypes.byref(tt), int(ignore_index),
+                                 _RED[reduction], ctypes.byref(tl),
+                                 ctypes.byref(tgX) if tgX is not None else None,
+                                 ctypes.byref(tgW) if tgW is not None else None,
+                                 B.stream_handle(stream), ctypes.byref(o), ctypes.byref(st))
+    B.check(rc, "flce_fwd_bwd_ex")
+    if host:
+        loss = loss.to("cpu", non_blocking=False)
+        gX = gX.cpu() if gX is not None else None
+        gW = gW.cpu() if gW is not None else None
+    res = (loss, gX, gW)
+    return res + (st.as_dict(),) if return_stats else res
+
+
+def cross_entropy(logits: torch.Tensor, target: torch.Tensor, ignore_index: int = -100,
+                  reduction: str = "mean", want_grad: bool = True, inplace: bool = False,
+                  n_valid: Optional[torch.Tensor] = None, row_loss: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, stream=None):
+    """Cross-entropy of given logits [BT, V]; the gradient may replace the logits in place."""
+    loss = torch.empty((), dtype=torch.float32, device=logits.device)
+    grad = None
+    if want_grad:
+        grad = logits if inplace else torch.empty_strided(logits.size(), logits.stride(), dtype=logits.dtype,
+                                                          device=logits.device)
+    o = _options(n_valid=n_valid, row_loss=row_loss, lse=lse)
+    tz, tt, tl = B.tensor(logits), B.tensor(target), B.tensor(loss)
+    tg = B.tensor(grad) if grad is not None else None
+    rc = B.lib().flce_cross_entropy(ctypes.byref(tz), ctypes.byref(tt), int(ignore_index), _RED[reduction],
+                                    ctypes.byref(tl), ctypes.byref(tg) if tg is not None else None,
+                                    B.stream_handle(stream), ctypes.byref(o))
+    B.check(rc, "flce_cross_entropy")
+    return loss, grad
+
+
+def count_valid(target: torch.Tensor, V: int, ignore_index: int = -100, stream=None) -> torch.Tensor:
+    """N (int64 device scalar): rows whose target is not ignore_index."""
+    n = torch.empty((), dtype=torch.int64, device=target.device)
+    tt = B.tensor(target)
+    B.check(B.lib().flce_count_valid(ctypes.byref(tt), int(V), int(ignore_index), B.ptr(n),
+                                     B.stream_handle(stream)), "flce_count_valid")
+    return n
+
+
+def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, M: int, N: int, K: int, a_mn_major: bool,
+              b_mn_major: bool, stream=None) -> torch.Tensor:
+    """C[M,N] fp32 = sum_k A(m,k) B(n,k) on the tcgen05 engine (a test hook)."""
+    C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    rc = B.lib().flce_gemm_bf16(B.ptr(A), B.ptr(Bm), B.ptr(C), M, N, K, A.stride(0), Bm.stride(0),
+                                C.stride(0), int(a_mn_major), int(b_mn_major), B.stream_handle(stream))
+    B.check(rc, "flce_gemm_bf16")
+    return C
+
+
+def plan(BT: int, H: int, V: int, dtype: str = "bf16", want_grad_W: bool = True,
+         chunk_rows: int = 0, workspace_limit_bytes: int = 0, grad_w_accum: str = "output") -> dict:
+    """Chunk rows, chunk count and workspace bytes for a shape (host only)."""
+    o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum)
+    st = B.FlceStats()
+    rc = B.lib().flce_plan(BT, H, V, B.BF16 if dtype == "bf16" else B.F32, int(want_grad_W),
+                           ctypes.byref(o), ctypes.byref(st))
+    B.check(rc, "flce_plan")
+    return st.as_dict()
+
+
+def device_error(stream=None) -> int:
+    """Read and clear the device error word (synchronises the stream)."""
+    e = ctypes.c_uint32(0)
+    B.check(B.lib().flce_get_device_error(B.stream_handle(stream), ctypes.byref(e)), "flce_get_device_error")
+    return e.value
+
+
+def phase_times(reset: bool = True) -> dict:
+    """{phase name: (milliseconds, launches)} for calls made with FLAG_TIME_PHASES."""
+    ms = (ctypes.c_double * B.NUM_PHASES)()
+    cnt = (ctypes.c_int32 * B.NUM_PHASES)()
+    B.check(B.lib().flce_phase_times(ms, cnt, B.NUM_PHASES, int(reset)), "flce_phase_times")
+    return {B.PHASE_NAMES[i]: (ms[i], cnt[i]) for i in range(B.NUM_PHASES)}
+
+
+class _FLCEFunction(torch.autograd.Function):
+    """Forward computes the loss and both gradients at once (the gradients are
+    produced in the forward pass and handed back, scaled, in backward)."""
+
+    @staticmethod
+    def forward(ctx, weight, inp, target, ignore_index, reduction, grad_w_accum):
+        shape = inp.shape
+        X = inp.reshape(-1, shape[-1])
+        if X.stride(-1) != 1 or (X.stride(0) % 8 and X.dtype == torch.bfloat16):
+            X = X.contiguous()
+        loss, gX, gW = fused_linear_cross_entropy(
+            X, weight, target.reshape(-1), ignore_index=ignore_index, reduction=reduction,
+            want_grad_X=ctx.needs_input_grad[1], want_grad_W=ctx.needs_input_grad[0],
+            grad_w_accum=grad_w_accum)
+        ctx.save_for_backward(gX if gX is not None else torch.empty(0), gW if gW is not None else torch.empty(0))
+        ctx.has = (gX is not None, gW is not None)
+        ctx.shape = shape
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        gX, gW = ctx.saved_tensors
+        hx, hw = ctx.has
+        one = grad_out.numel() == 1 and bool(grad_out == 1)
+        dX = (gX if one else gX * grad_out.to(gX.dtype)).reshape(ctx.shape) if hx else None
+        dW = (gW if one else gW * grad_out.to(gW.dtype)) if hw else None
+        return dW, dX, None, None, None, None
+
+
+class FusedLinearCrossEntropyLoss(torch.nn.Module):
+    """loss_fn(lm_head.weight, input, target) -> scalar loss with autograd.
+
+    input may be [BT, H] or [B, T, H]; target has the matching leading shape.
+    """
+
+    def __init__(self, ignore_index: int = -100, reduction: str = "mean", grad_w_accum: str = "output"):
+        super().__init__()
+        if reduction not in _RED:
+            raise ValueError("reduction must be 'mean' or 'sum'")
+        self.ignore_index = ignore_index
+        self.reduction = reduction
+        self.grad_w_accum = grad_w_accum
+
+    def forward(self, weight, input, target):  # noqa: A002 - mirrors the pages' call
+        return _FLCEFunction.apply(weight, input, target, self.ignore_index, self.reduction, self.grad_w_accum)

@@ -1,0 +1,425 @@
+// Memory-bound steps of fused linear cross-entropy and the exact-fp32 SIMT path.
+//
+//   count_valid_kernel   N = #rows whose target is not ignore_index (A0)
+//   combine_kernel       per row: merge the per-tile (max, sum-exp) partials
+//                        into lse, write l_i = lse - z_t, and turn each tile's
+//                        max into the factor exp(m_tile - lse) * scale (A3)
+//   dlogits_kernel       in place over the chunk store: e * factor - onehot*scale,
+//                        0 for ignored rows (A4, "in-place gradient replacement"
+//                        of the paper review's 主な発見)
+//   finalize_loss_kernel fixed-order sum of the per-row losses, times 1/N or 1
+//   ce_partials_kernel   logits given: per-(row, tile) partials read from z
+//   ce_grad_kernel       logits given: dz from z and lse, optionally in place
+//   simt_gemm_kernel     fp32 FMA GEMM with the same epilogues as the tcgen05
+//                        engine, for fp32 inputs where TF32 tensor cores would
+//                        not meet an exact-fp32 tolerance
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace flce {
+
+__device__ __forceinline__ bool target_valid(int64_t t, int64_t V, int64_t ignore_index) {
+  return t != ignore_index && t >= 0 && t < V;
+}
+
+__device__ __forceinline__ float mean_scale(const int64_t* n_valid, int reduction) {
+  if (reduction != 0) return 1.f;
+  const int64_t n = *n_valid;
+  return n > 0 ? 1.f / (float)n : 0.f;
+}
+
+// ------------------------------------------------------------------ A0
+// One block; integer counts, so the order of the reduction does not matter.
+__global__ void count_valid_kernel(const int64_t* __restrict__ target, int64_t BT, int64_t V,
+                                   int64_t ignore_index, int64_t* n_valid, uint32_t* err) {
+  __shared__ unsigned long long part[32];
+  unsigned long long c = 0;
+  bool bad = false;
+  for (int64_t i = threadIdx.x; i < BT; i += blockDim.x) {
+    const int64_t t = target[i];
+    if (t == ignore_index) continue;
+    if (t >= 0 && t < V) ++c; else bad = true;
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(err, DEVERR_TARGET_RANGE);
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    c = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0ull;
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (threadIdx.x == 0) *n_valid = (int64_t)c;
+  }
+}
+
+// ------------------------------------------------------------------ A3
+// Block = 256 threads = 8 warps over 32 rows: lane <-> row, warp w merges
+// tiles w, w+8, ... so every partial load is a coalesced 128-byte read.
+struct CombineArgs {
+  const int64_t* target;  // chunk row 0
+  int64_t ignore_index, V;
+  int rows;               // rows in this chunk
+  int ntile;              // partial tiles per row
+  int64_t ldp;
+  float* part_m;          // in: tile max; out: exp(m_tile - lse) * scale (0 for ignored rows)
+  const float* part_s;
+  const float* zt;
+  float* row_loss;        // [rows] at chunk row 0: l_i (0 for ignored rows)
+  float* lse_out;         // optional [rows] at chunk row 0
+  const int64_t* n_valid;
+  int reduction;
+};
+
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  __shared__ float sm_m[8][32], sm_s[8][32], sm_lse[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int r = blockIdx.x * 32 + lane;
+  const bool row_ok = r < a.rows;
+  float M = -INFINITY, S = 0.f;
+  if (row_ok) {
+    for (int j = w; j < a.ntile; j += 8) {
+      const float m = a.part_m[(int64_t)j * a.ldp + r];
+      const float s = a.part_s[(int64_t)j * a.ldp + r];
+      if (m > M) {
+        S = S * exp2f((M - m) * LOG2E_F) + s;
+        M = m;
+      } else {
+        S += s * exp2f((m - M) * LOG2E_F);
+      }
+    }
+  }
+  sm_m[w][lane] = M;
+  sm_s[w][lane] = S;
+  __syncthreads();
+  if (w == 0) {
+    float Mt = -INFINITY;
+    for (int k = 0; k < 8; ++k) Mt = fmaxf(Mt, sm_m[k][lane]);
+    float St = 0.f;
+    for (int k = 0; k < 8; ++k)
+      if (sm_m[k][lane] != -INFINITY) St += sm_s[k][lane] * exp2f((sm_m[k][lane] - Mt) * LOG2E_F);
+    const float lse = Mt + logf(St);
+    sm_lse[lane] = lse;
+    if (row_ok) {
+      const int64_t t = a.target[r];
+      const bool valid = target_valid(t, a.V, a.ignore_index);
+      a.row_loss[r] = valid ? lse - a.zt[r] : 0.f;
+      if (a.lse_out) a.lse_out[r] = lse;
+    }
+  }
+  __syncthreads();
+  if (row_ok) {
+    const bool valid = target_valid(a.target[r], a.V, a.ignore_index);
+    const float scale = mean_scale(a.n_valid, a.reduction);
+    const float lse = sm_lse[lane];
+    for (int j = w; j < a.ntile; j += 8) {
+      float* pm = a.part_m + (int64_t)j * a.ldp + r;
+      *pm = valid ? exp2f((*pm - lse) * LOG2E_F) * scale : 0.f;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ A4
+// grid.y = chunk row, grid.x * blockDim.x covers the row in vectors of 8.
+template <typename T>
+struct Vec8;
+template <>
+struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x = unpack_bf16x2(w[k]);
+      f[2 * k] = x.x;
+      f[2 * k + 1] = x.y;
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&f)[8]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                              pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+  }
+  static __device__ __forceinline__ float ld1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ void st1(__nv_bfloat16* p, float f) { *p = __float2bfloat16_rn(f); }
+};
+template <>
+struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&f)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&f)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+  static __device__ __forceinline__ float ld1(const float* p) { return *p; }
+  static __device__ __forceinline__ void st1(float* p, float f) { *p = f; }
+};
+
+template <typename T>
+struct DlogitsArgs {
+  T* e;                   // [rows, lde] in: exp(z - m_tile); out: dz
+  int64_t lde;
+  const T* src;           // where e is read from (== e for in place)
+  int64_t lds;
+  const int64_t* target;  // chunk row 0
+  int64_t ignore_index, V;
+  const float* factor;    // [ntile, ldp]
+  int64_t ldp;
+  int tile_shift;         // log2 of the partial tile width
+  const int64_t* n_valid;
+  int reduction;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs<T> a) {
+  const int64_t r = blockIdx.y;
+  const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (c0 >= a.V) return;
+  const int64_t t = a.target[r];
+  const bool valid = target_valid(t, a.V, a.ignore_index);
+  const float scale = mean_scale(a.n_valid, a.reduction);
+  const float f = a.factor[(c0 >> a.tile_shift) * a.ldp + r];
+  const T* s = a.src + r * a.lds + c0;
+  T* d = a.e + r * a.lde + c0;
+  float v[8];
+  const bool full = c0 + 8 <= a.V;
+  if (full) {
+    Vec8<T>::load(s, v);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = c0 + k < a.V ? Vec8<T>::ld1(s + k) : 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float x = valid ? v[k] * f : 0.f;
+    if (valid && c0 + k == t) x -= scale;
+    v[k] = x;
+  }
+  if (full) {
+    Vec8<T>::store(d, v);
+  } else {
+    for (int k = 0; k < 8 && c0 + k < a.V; ++k) Vec8<T>::st1(d + k, v[k]);
+  }
+}
+
+// Logits-given cross-entropy, pass 1: the per-(row, tile) (max, sum-exp)
+// partials and the target logit, one warp per (row, tile of 1 << tile_shift).
+template <typename T>
+struct CePartialArgs {
+  const T* z;
+  int64_t ldz;
+  const int64_t* target;
+  int64_t ignore_index, V;
+  float* part_m;
+  float* part_s;
+  int64_t ldp;
+  float* zt;
+  int rows, ntile, tile_shift;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) ce_partials_kernel(CePartialArgs<T> a) {
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t r = warp_global / a.ntile;
+  const int j = (int)(warp_global % a.ntile);
+  if (r >= a.rows) return;
+  const int64_t n0 = (int64_t)j << a.tile_shift;
+  const int64_t n1 = (n0 + (1 << a.tile_shift)) < a.V ? (n0 + (1 << a.tile_shift)) : a.V;
+  const T* zr = a.z + r * a.ldz;
+  float m = -INFINITY;
+  for (int64_t c = n0 + lane; c < n1; c += 32) m = fmaxf(m, Vec8<T>::ld1(zr + c));
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float ms = m * LOG2E_F;
+  float s = 0.f;
+  for (int64_t c = n0 + lane; c < n1; c += 32) s += exp2f(fmaf(Vec8<T>::ld1(zr + c), LOG2E_F, -ms));
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    a.part_m[(int64_t)j * a.ldp + r] = m;
+    a.part_s[(int64_t)j * a.ldp + r] = s;
+    const int64_t t = a.target[r];
+    if (t != a.ignore_index && t >= n0 && t < n1) a.zt[r] = Vec8<T>::ld1(zr + t);
+  }
+}
+
+// Logits-given cross-entropy, pass 2: dz = (exp(z - lse) - onehot) * scale,
+// 0 for ignored rows; dst may be z itself (in-place gradient replacement).
+template <typename T>
+struct CeGradArgs {
+  const T* z;
+  int64_t ldz;
+  T* dz;
+  int64_t ldd;
+  const int64_t* target;
+  int64_t ignore_index, V;
+  const float* lse;
+  const int64_t* n_valid;
+  int reduction;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) ce_grad_kernel(CeGradArgs<T> a) {
+  const int64_t r = blockIdx.y;
+  const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (c0 >= a.V) return;
+  const int64_t t = a.target[r];
+  const bool valid = target_valid(t, a.V, a.ignore_index);
+  const float scale = mean_scale(a.n_valid, a.reduction);
+  const float ls = a.lse[r] * LOG2E_F;
+  const T* s = a.z + r * a.ldz + c0;
+  T* d = a.dz + r * a.ldd + c0;
+  const bool full = c0 + 8 <= a.V;
+  float v[8];
+  if (full) {
+    Vec8<T>::load(s, v);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = c0 + k < a.V ? Vec8<T>::ld1(s + k) : 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float x = valid ? exp2f(fmaf(v[k], LOG2E_F, -ls)) * scale : 0.f;
+    if (valid && c0 + k == t) x -= scale;
+    v[k] = x;
+  }
+  if (full) {
+    Vec8<T>::store(d, v);
+  } else {
+    for (int k = 0; k < 8 && c0 + k < a.V; ++k) Vec8<T>::st1(d + k, v[k]);
+  }
+}
+
+// ------------------------------------------------------------------ loss
+// One block, fixed order: thread k sums rows k, k+1024, ... in double, then a
+// fixed shuffle tree. Deterministic for a given BT.
+__global__ void __launch_bounds__(1024) finalize_loss_kernel(const float* __restrict__ row_loss,
+                                                             int64_t BT, const int64_t* n_valid,
+                                                             int reduction, float* loss) {
+  __shared__ double part[32];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < BT; i += blockDim.x) acc += (double)row_loss[i];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    acc = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.0;
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (threadIdx.x == 0) {
+      if (reduction == 0) {
+        const int64_t n = *n_valid;
+        *loss = n > 0 ? (float)(acc / (double)n) : 0.f;
+      } else {
+        *loss = (float)acc;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ SIMT fp32
+// C(m, n) = sum_k A(m, k) * B(n, k) with A(m, k) = A[m*sam + k*sak] and
+// B(n, k) = B[n*sbn + k*sbk]. 64 x 64 tiles, 256 threads, 4 x 4 per thread.
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
+
+enum SimtEpi : int { SEPI_LOGITS = 0, SEPI_STORE = 1, SEPI_GRADW_STORE = 2, SEPI_GRADW_ADD = 3 };
+
+struct SimtArgs {
+  const float* A;
+  int64_t sam, sak;
+  const float* B;
+  int64_t sbn, sbk;
+  int M, N, K;
+  int epi;
+  float* out;
+  int64_t ldo;
+  // SEPI_LOGITS
+  const int64_t* target;
+  int64_t ignore_index;
+  float* part_m;
+  float* part_s;
+  int64_t ldp;
+  float* zt;
+};
+
+__global__ void __launch_bounds__(256) simt_gemm_kernel(SimtArgs a) {
+  __shared__ float As[SG_BK][SG_BM + 4];
+  __shared__ float Bs[SG_BK][SG_BN + 4];
+  __shared__ float Cs[SG_BM][SG_BN + 1];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int64_t m0 = (int64_t)blockIdx.y * SG_BM, n0 = (int64_t)blockIdx.x * SG_BN;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < a.K; k0 += SG_BK) {
+    for (int i = tid; i < SG_BM * SG_BK; i += 256) {
+      int mm, kk;
+      if (a.sak == 1) { mm = i / SG_BK; kk = i % SG_BK; } else { kk = i / SG_BM; mm = i % SG_BM; }
+      const int64_t gm = m0 + mm, gk = k0 + kk;
+      As[kk][mm] = (gm < a.M && gk < a.K) ? a.A[gm * a.sam + gk * a.sak] : 0.f;
+    }
+    for (int i = tid; i < SG_BN * SG_BK; i += 256) {
+      int nn, kk;
+      if (a.sbk == 1) { nn = i / SG_BK; kk = i % SG_BK; } else { kk = i / SG_BN; nn = i % SG_BN; }
+      const int64_t gn = n0 + nn, gk = k0 + kk;
+      Bs[kk][nn] = (gn < a.N && gk < a.K) ? a.B[gn * a.sbn + gk * a.sbk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  if (a.epi != SEPI_LOGITS) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t gm = m0 + ty * 4 + i;
+      if (gm >= a.M) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t gn = n0 + tx * 4 + j;
+        if (gn >= a.N) continue;
+        float* o = a.out + gm * a.ldo + gn;
+        *o = a.epi == SEPI_GRADW_ADD ? *o + acc[i][j] : acc[i][j];
+      }
+    }
+    return;
+  }
+  // online-softmax epilogue over this 64-column tile: one thread per row
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) Cs[ty * 4 + i][tx * 4 + j] = acc[i][j];
+  __syncthreads();
+  if (tid < SG_BM) {
+    const int64_t r = m0 + tid;
+    if (r >= a.M) return;
+    const int ncols = (int)((a.N - n0) < SG_BN ? (a.N - n0) : SG_BN);
+    float mx = -INFINITY;
+    for (int j = 0; j < ncols; ++j) mx = fmaxf(mx, Cs[tid][j]);
+    const float ms = mx * LOG2E_F;
+    float s = 0.f;
+    float* er = a.out + r * a.ldo + n0;
+    for (int j = 0; j < ncols; ++j) {
+      const float e = exp2f(fmaf(Cs[tid][j], LOG2E_F, -ms));
+      s += e;
+      er[j] = e;
+    }
+    const int64_t tile = blockIdx.x;
+    a.part_m[tile * a.ldp + r] = mx;
+    a.part_s[tile * a.ldp + r] = s;
+    const int64_t t = a.target[r];
+    if (t != a.ignore_index && t >= n0 && t < n0 + ncols) a.zt[r] = Cs[tid][t - n0];
+  }
+}
+
+}  // namespace flce

@@ -1,0 +1,744 @@
+// Host side of the fused linear cross-entropy library: argument checks, the
+// bounded-workspace chunk plan, TMA descriptors, and the launch sequence.
+//
+// Per chunk of rows (the "chunking" of "Liger Kernel: Efficient Triton Kernels
+// for LLM Training", paper review, 提案手法; and of "Liger-Kernel 項目詳細介紹",
+// 技術原理 > 分塊計算):
+//   A1+A2  logits GEMM z = X_c W^T with the online-softmax epilogue
+//   A3     row combine: lse, per-row loss, per-tile factors
+//   A4     in-place dlogits over the chunk store (技術原理 > 原地操作)
+//   A5+A6  grad_X_c = dz W and grad_W (+)= dz^T X_c in one persistent launch
+// then one fixed-order loss reduction. The full BT x V logits never exist:
+// the store holds one chunk of rows at a time.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/flce.h"
+#include "aux_kernels.cuh"
+#include "tc_gemm.cuh"
+
+namespace flce {
+
+__device__ uint32_t g_err_word;  // device error word (FLCE_DEVERR_* bits), one per device
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kDefaultLimit = 512ll << 20;
+constexpr int64_t kMaxChunk = 32768;
+
+struct DeviceCtx {
+  bool init = false;
+  bool supported = false;
+  int sms = 0;
+  uint32_t* err = nullptr;
+};
+
+std::mutex g_mu;
+DeviceCtx g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+struct PhaseRec {
+  int phase;
+  cudaEvent_t a, b;
+};
+std::vector<PhaseRec> g_phase_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+flce_status device_ctx(DeviceCtx** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FLCE_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceCtx& c = g_dev[dev];
+  if (!c.init) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FLCE_ERR_CUDA;
+    c.supported = prop.major == 10 && prop.minor == 0;
+    c.sms = prop.multiProcessorCount;
+    if (c.supported) {
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.err), g_err_word) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+      if (cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               TC_SMEM_BYTES) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+      if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+          return FLCE_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      }
+    }
+    c.init = true;
+  }
+  if (!c.supported) return FLCE_ERR_UNSUPPORTED_DEVICE;
+  *out = &c;
+  return FLCE_OK;
+}
+
+// bf16 2-D tensor map: dims {inner, outer}, row pitch in bytes, box {bi, bo}, 128B swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t pitch_bytes, uint32_t bi, uint32_t bo) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {bi, bo};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int dtype_size(int32_t dt) { return dt == FLCE_F32 ? 4 : dt == FLCE_BF16 ? 2 : dt == FLCE_I64 ? 8 : 0; }
+
+bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// A row-major matrix of the given shape and dtype.
+bool check_matrix(const flce_tensor* t, int32_t dtype, int64_t rows, int64_t cols) {
+  if (!t || !t->data || t->dtype != dtype || t->ndim != 2) return false;
+  if (t->shape[0] != rows || t->shape[1] != cols) return false;
+  if (t->stride[1] != 1 || t->stride[0] < cols) return false;
+  return true;
+}
+
+struct Plan {
+  int64_t BT, H, V;
+  int32_t dtype;
+  int64_t chunk, n_chunks;
+  int64_t tile_w;  // partial tile width (columns)
+  int64_t ntile, lde, ldp;
+  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, total;
+  bool facc;
+};
+
+flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want_gw,
+                      const flce_options* opt, bool need_rowloss, Plan* p) {
+  if (BT < 0 || H <= 0 || V <= 0) return FLCE_ERR_INVALID_ARG;
+  if (dtype != FLCE_BF16 && dtype != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
+  p->BT = BT;
+  p->H = H;
+  p->V = V;
+  p->dtype = dtype;
+  const int64_t esz = dtype == FLCE_BF16 ? 2 : 4;
+  p->tile_w = dtype == FLCE_BF16 ? TC_BN : SG_BN;
+  p->ntile = ceil_div(V, p->tile_w);
+  p->lde = round_up(V, 64);
+  const int64_t per_row = p->lde * esz + p->ntile * 8 + 4;
+  int64_t chunk = opt && opt->chunk_rows > 0 ? round_up(opt->chunk_rows, 128) : 0;
+  const int64_t bt_r = std::max<int64_t>(round_up(std::max<int64_t>(BT, 1), 128), 128);
+  if (chunk == 0) {
+    if (opt && opt->workspace_limit_bytes > 0) {
+      chunk = (opt->workspace_limit_bytes / per_row) / 128 * 128;
+    } else {
+      // default: at most 512 MiB of chunk store, and at most half of the rows,
+      // so the logits of the whole batch are never held at once
+      chunk = std::min<int64_t>((kDefaultLimit / per_row) / 128 * 128,
+                                round_up(ceil_div(std::max<int64_t>(BT, 1), 2), 128));
+    }
+    if (chunk < 128) chunk = 128;
+    if (chunk > kMaxChunk) chunk = kMaxChunk;
+    // even out the chunks: same count, rows spread as evenly as 128-row tiles allow
+    if (BT > 0) chunk = round_up(ceil_div(BT, ceil_div(BT, chunk)), 128);
+  }
+  if (chunk > bt_r) chunk = bt_r;
+  if (chunk > kMaxChunk) chunk = kMaxChunk;  // grid.y of the row kernels stays below 65536
+  p->chunk = chunk;
+  p->n_chunks = BT > 0 ? ceil_div(BT, chunk) : 0;
+  p->ldp = round_up(chunk, 32);
+  p->facc = want_gw && dtype == FLCE_BF16 && opt && opt->grad_w_accum == FLCE_GRADW_ACCUM_FP32 &&
+            p->n_chunks > 1;
+  size_t o = 0;
+  p->off_nvalid = o; o = align256(o + 8);
+  p->off_rowloss = o; o = align256(o + (need_rowloss ? (size_t)std::max<int64_t>(BT, 1) * 4 : 0));
+  p->off_zt = o; o = align256(o + (size_t)chunk * 4);
+  p->off_pm = o; o = align256(o + (size_t)p->ntile * p->ldp * 4);
+  p->off_ps = o; o = align256(o + (size_t)p->ntile * p->ldp * 4);
+  p->off_e = o; o = align256(o + (size_t)chunk * p->lde * esz);
+  p->off_facc = o; o = align256(o + (p->facc ? (size_t)V * H * 4 : 0));
+  p->total = o;
+  return FLCE_OK;
+}
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launch bookkeeping: optional phase events, launch-error checks, counts.
+struct Launcher {
+  cudaStream_t stream;
+  bool timing, sync_check;
+  int launches = 0;
+  template <typename F>
+  flce_status run(int phase, F&& f) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (timing) {
+      std::lock_guard<std::mutex> lk(g_mu);
+      a = pool_event();
+      b = pool_event();
+    }
+    if (a) cudaEventRecord(a, stream);
+    f();
+    ++launches;
+    if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    if (b) {
+      cudaEventRecord(b, stream);
+      std::lock_guard<std::mutex> lk(g_mu);
+      g_phase_recs.push_back({phase, a, b});
+    }
+    if (sync_check) {
+      if (cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+      if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+    }
+    return FLCE_OK;
+  }
+};
+
+bool env_debug() {
+  const char* s = std::getenv("FLCE_DEBUG");
+  return s && s[0] && s[0] != '0';
+}
+
+// Workspace holder: caller's buffer or a stream-ordered allocation.
+struct Workspace {
+  void* ptr = nullptr;
+  bool owned = false;
+  cudaStream_t stream = nullptr;
+  ~Workspace() {
+    if (owned && ptr) cudaFreeAsync(ptr, stream);
+  }
+};
+
+flce_status get_workspace(const flce_options* opt, size_t bytes, cudaStream_t stream,
+                          Workspace* ws) {
+  ws->stream = stream;
+  if (opt && opt->workspace) {
+    if ((size_t)opt->workspace_bytes < bytes) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+    if (!is_aligned(opt->workspace, 256)) return FLCE_ERR_INVALID_ARG;
+    ws->ptr = opt->workspace;
+    return FLCE_OK;
+  }
+  if (cudaMallocAsync(&ws->ptr, bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    ws->ptr = nullptr;
+    return FLCE_ERR_ALLOC;
+  }
+  ws->owned = true;
+  return FLCE_OK;
+}
+
+TcProblem make_problem(int M, int N, int K, int a_mn, int b_mn, int epi, int m_fastest) {
+  TcProblem P;
+  std::memset(&P, 0, sizeof(P));
+  P.M = M;
+  P.N = N;
+  P.K = K;
+  P.tiles_m = (int)ceil_div(M, TC_BM);
+  P.tiles_n = (int)ceil_div(N, TC_BN);
+  P.kblocks = (int)ceil_div(K, TC_BK);
+  P.a_mn = a_mn;
+  P.b_mn = b_mn;
+  P.epi = epi;
+  P.m_fastest = m_fastest;
+  return P;
+}
+
+void launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+               const CUtensorMap& b1, const TcParams& prm, int sms, cudaStream_t stream) {
+  int64_t tiles = (int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n;
+  if (prm.nprob > 1) tiles += (int64_t)prm.prob[1].tiles_m * prm.prob[1].tiles_n;
+  const int grid = (int)std::min<int64_t>(sms, tiles);
+  tc_gemm_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
+}
+
+// ------------------------------------------------------------------ FLCE
+flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tensor* target,
+                     int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                     flce_tensor* grad_X, flce_tensor* grad_W, cudaStream_t stream,
+                     const flce_options* opt, flce_stats* stats) {
+  // ---- host-side argument checks (nothing is enqueued before they pass)
+  if (!X || !W || !target || !loss) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_MEAN && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  const int32_t dt = X->dtype;
+  if (dt != FLCE_BF16 && dt != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
+  if (W->dtype != dt) return FLCE_ERR_UNSUPPORTED_DTYPE;
+  if (X->ndim != 2 || W->ndim != 2) return FLCE_ERR_INVALID_ARG;
+  const int64_t BT = X->shape[0], H = X->shape[1], V = W->shape[0];
+  if (BT < 0 || H <= 0 || V <= 0 || W->shape[1] != H) return FLCE_ERR_INVALID_ARG;
+  if (BT >= (1ll << 31) || V >= (1ll << 31) || H >= (1ll << 31)) return FLCE_ERR_INVALID_ARG;
+  if ((BT > 0 && !check_matrix(X, dt, BT, H)) || !check_matrix(W, dt, V, H)) return FLCE_ERR_INVALID_ARG;
+  if (target->dtype != FLCE_I64 || target->ndim != 1 || target->shape[0] != BT ||
+      (BT > 0 && (!target->data || target->stride[0] != 1)))
+    return FLCE_ERR_INVALID_ARG;
+  if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
+      (loss->ndim == 1 && loss->shape[0] != 1))
+    return FLCE_ERR_INVALID_ARG;
+  if (grad_X && (BT > 0 && !check_matrix(grad_X, dt, BT, H))) return FLCE_ERR_INVALID_ARG;
+  if (grad_W && !check_matrix(grad_W, dt, V, H)) return FLCE_ERR_INVALID_ARG;
+  if (dt == FLCE_BF16) {
+    // TMA and 16-byte vector stores: 16-byte aligned bases and rows
+    if (H % 8 || !is_aligned(W->data, 16) || W->stride[0] % 8) return FLCE_ERR_INVALID_ARG;
+    if (BT > 0 && (!is_aligned(X->data, 16) || X->stride[0] % 8)) return FLCE_ERR_INVALID_ARG;
+    if (grad_X && BT > 0 && (!is_aligned(grad_X->data, 16) || grad_X->stride[0] % 8)) return FLCE_ERR_INVALID_ARG;
+    if (grad_W && (!is_aligned(grad_W->data, 16) || grad_W->stride[0] % 8)) return FLCE_ERR_INVALID_ARG;
+  }
+  const bool want_gx = grad_X != nullptr && BT > 0;
+  const bool want_gw = grad_W != nullptr;
+  const bool need_rowloss = !(opt && opt->row_loss);
+  Plan pl;
+  flce_status st = make_plan(BT, H, V, dt, want_gw, opt, need_rowloss, &pl);
+  if (st != FLCE_OK) return st;
+
+  DeviceCtx* dev = nullptr;
+  st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+
+  Launcher L{stream, opt && (opt->flags & FLCE_FLAG_TIME_PHASES), env_debug() || (opt && (opt->flags & FLCE_FLAG_SYNC_CHECK))};
+  if (stats) {
+    std::memset(stats, 0, sizeof(*stats));
+    stats->chunk_rows = pl.chunk;
+    stats->n_chunks = pl.n_chunks;
+    stats->workspace_bytes = (int64_t)pl.total;
+    stats->materialized_logits_bytes = BT * V * 2;
+    stats->path = dt == FLCE_BF16 ? 1 : 0;
+  }
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+
+  if (BT == 0) {
+    if (cudaMemsetAsync(loss->data, 0, 4, stream) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (want_gw && cudaMemset2DAsync(grad_W->data, grad_W->stride[0] * dtype_size(dt), 0,
+                                     H * dtype_size(dt), V, stream) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    if (stats) stats->workspace_bytes = 0;
+    return FLCE_OK;
+  }
+
+  Workspace ws;
+  st = get_workspace(opt, pl.total, stream, &ws);
+  if (st != FLCE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws.ptr);
+  int64_t* nvalid_local = reinterpret_cast<int64_t*>(base + pl.off_nvalid);
+  const int64_t* nvalid = (opt && opt->n_valid) ? opt->n_valid : nvalid_local;
+  float* row_loss = need_rowloss ? reinterpret_cast<float*>(base + pl.off_rowloss) : opt->row_loss;
+  float* zt = reinterpret_cast<float*>(base + pl.off_zt);
+  float* pm = reinterpret_cast<float*>(base + pl.off_pm);
+  float* ps = reinterpret_cast<float*>(base + pl.off_ps);
+  void* estore = base + pl.off_e;
+  float* facc = pl.facc ? reinterpret_cast<float*>(base + pl.off_facc) : nullptr;
+  float* lse_out = opt ? opt->lse : nullptr;
+  const int64_t* tgt = static_cast<const int64_t*>(target->data);
+
+  // A0: N (always run: it also flags targets outside [0, V))
+  st = L.run(0, [&] {
+    count_valid_kernel<<<1, 1024, 0, stream>>>(tgt, BT, V, ignore_index, nvalid_local, dev->err);
+  });
+  if (st != FLCE_OK) return st;
+
+  const int64_t ldx = X->stride[0], ldw = W->stride[0];
+  for (int64_t c = 0; c < pl.n_chunks; ++c) {
+    const int64_t r0 = c * pl.chunk;
+    const int rows = (int)std::min<int64_t>(pl.chunk, BT - r0);
+    const int64_t* tgt_c = tgt + r0;
+    if (dt == FLCE_BF16) {
+      const __nv_bfloat16* Xc = static_cast<const __nv_bfloat16*>(X->data) + r0 * ldx;
+      const __nv_bfloat16* Wp = static_cast<const __nv_bfloat16*>(W->data);
+      __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
+      // A1 + A2
+      {
+        CUtensorMap ta, tb, z;
+        std::memset(&z, 0, sizeof(z));
+        if (!make_tmap(&ta, Xc, H, rows, ldx * 2, 64, TC_BM) || !make_tmap(&tb, Wp, H, V, ldw * 2, 64, TC_BN))
+          return FLCE_ERR_CUDA;
+        TcParams prm;
+        std::memset(&prm, 0, sizeof(prm));
+        prm.nprob = 1;
+        prm.prob[0] = make_problem(rows, (int)V, (int)H, 0, 0, EPI_LOGITS, 1);
+        prm.lg = LogitsArgs{tgt_c, ignore_index, V, E, pl.lde, pm, ps, pl.ldp, zt};
+        prm.err = dev->err;
+        st = L.run(1, [&] { launch_tc(ta, tb, z, z, prm, dev->sms, stream); });
+        if (st != FLCE_OK) return st;
+      }
+    } else {
+      SimtArgs s;
+      std::memset(&s, 0, sizeof(s));
+      s.A = static_cast<const float*>(X->data) + r0 * ldx; s.sam = ldx; s.sak = 1;
+      s.B = static_cast<const float*>(W->data); s.sbn = ldw; s.sbk = 1;
+      s.M = rows; s.N = (int)V; s.K = (int)H;
+      s.epi = SEPI_LOGITS;
+      s.out = static_cast<float*>(estore); s.ldo = pl.lde;
+      s.target = tgt_c; s.ignore_index = ignore_index;
+      s.part_m = pm; s.part_s = ps; s.ldp = pl.ldp; s.zt = zt;
+      st = L.run(1, [&] {
+        simt_gemm_kernel<<<dim3((unsigned)ceil_div(V, SG_BN), (unsigned)ceil_div(rows, SG_BM)), 256, 0, stream>>>(s);
+      });
+      if (st != FLCE_OK) return st;
+    }
+    // A3
+    {
+      CombineArgs a{tgt_c, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, ps, zt,
+                    row_loss + r0, lse_out ? lse_out + r0 : nullptr, nvalid, reduction};
+      st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
+      if (st != FLCE_OK) return st;
+    }
+    if (!want_gx && !want_gw) continue;
+    // A4
+    {
+      const int shift = dt == FLCE_BF16 ? 8 : 6;
+      const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
+      if (dt == FLCE_BF16) {
+        __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
+        DlogitsArgs<__nv_bfloat16> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction};
+        st = L.run(3, [&] { dlogits_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a); });
+      } else {
+        float* E = static_cast<float*>(estore);
+        DlogitsArgs<float> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction};
+        st = L.run(3, [&] { dlogits_kernel<float><<<grid, 256, 0, stream>>>(a); });
+      }
+      if (st != FLCE_OK) return st;
+    }
+    // A5 + A6
+    if (dt == FLCE_BF16) {
+      const __nv_bfloat16* Xc = static_cast<const __nv_bfloat16*>(X->data) + r0 * ldx;
+      const __nv_bfloat16* Wp = static_cast<const __nv_bfloat16*>(W->data);
+      __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
+      CUtensorMap tm[4];
+      std::memset(tm, 0, sizeof(tm));
+      TcParams prm;
+      std::memset(&prm, 0, sizeof(prm));
+      prm.err = dev->err;
+      int np = 0;
+      if (want_gx) {
+        if (!make_tmap(&tm[2 * np], E, V, rows, pl.lde * 2, 64, TC_BM) ||
+            !make_tmap(&tm[2 * np + 1], Wp, H, V, ldw * 2, 64, 64))
+          return FLCE_ERR_CUDA;
+        TcProblem P = make_problem(rows, (int)H, (int)V, 0, 1, EPI_STORE_BF16, 1);
+        P.out = static_cast<__nv_bfloat16*>(grad_X->data) + r0 * grad_X->stride[0];
+        P.ldo = grad_X->stride[0];
+        prm.prob[np++] = P;
+      }
+      if (want_gw) {
+        if (!make_tmap(&tm[2 * np], E, V, rows, pl.lde * 2, 64, 64) ||
+            !make_tmap(&tm[2 * np + 1], Xc, H, rows, ldx * 2, 64, 64))
+          return FLCE_ERR_CUDA;
+        TcProblem P = make_problem((int)V, (int)H, rows, 1, 1, EPI_GRADW, 0);
+        P.out = grad_W->data;
+        P.ldo = grad_W->stride[0];
+        const bool last = c == pl.n_chunks - 1;
+        if (!pl.facc) P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
+        else P.gw_mode = c == 0 ? GW_STORE_F32 : (last ? GW_FINAL_F32 : GW_ADD_F32);
+        P.facc = facc;
+        P.ld_facc = H;
+        prm.prob[np++] = P;
+      }
+      prm.nprob = np;
+      st = L.run(4, [&] { launch_tc(tm[0], tm[1], tm[2], tm[3], prm, dev->sms, stream); });
+      if (st != FLCE_OK) return st;
+    } else {
+      float* E = static_cast<float*>(estore);
+      if (want_gx) {
+        SimtArgs s;
+        std::memset(&s, 0, sizeof(s));
+        s.A = E; s.sam = pl.lde; s.sak = 1;
+        s.B = static_cast<const float*>(W->data); s.sbn = 1; s.sbk = ldw;
+        s.M = rows; s.N = (int)H; s.K = (int)V;
+        s.epi = SEPI_STORE;
+        s.out = static_cast<float*>(grad_X->data) + r0 * grad_X->stride[0];
+        s.ldo = grad_X->stride[0];
+        st = L.run(4, [&] {
+          simt_gemm_kernel<<<dim3((unsigned)ceil_div(H, SG_BN), (unsigned)ceil_div(rows, SG_BM)), 256, 0, stream>>>(s);
+        });
+        if (st != FLCE_OK) return st;
+      }
+      if (want_gw) {
+        SimtArgs s;
+        std::memset(&s, 0, sizeof(s));
+        s.A = E; s.sam = 1; s.sak = pl.lde;
+        s.B = static_cast<const float*>(X->data) + r0 * ldx; s.sbn = 1; s.sbk = ldx;
+        s.M = (int)V; s.N = (int)H; s.K = rows;
+        s.epi = c == 0 ? SEPI_GRADW_STORE : SEPI_GRADW_ADD;
+        s.out = static_cast<float*>(grad_W->data);
+        s.ldo = grad_W->stride[0];
+        st = L.run(4, [&] {
+          simt_gemm_kernel<<<dim3((unsigned)ceil_div(H, SG_BN), (unsigned)ceil_div(V, SG_BM)), 256, 0, stream>>>(s);
+        });
+        if (st != FLCE_OK) return st;
+      }
+    }
+  }
+  st = L.run(5, [&] {
+    finalize_loss_kernel<<<1, 1024, 0, stream>>>(row_loss, BT, nvalid, reduction,
+                                                 static_cast<float*>(loss->data));
+  });
+  if (st != FLCE_OK) return st;
+  if (stats) stats->kernel_launches = L.launches;
+  return FLCE_OK;
+}
+
+// ------------------------------------------------------------------ CE (logits given)
+flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t ignore_index,
+                   int32_t reduction, flce_tensor* loss, flce_tensor* grad, cudaStream_t stream,
+                   const flce_options* opt) {
+  if (!Z || !target || !loss) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_MEAN && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  const int32_t dt = Z->dtype;
+  if (dt != FLCE_BF16 && dt != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
+  if (Z->ndim != 2) return FLCE_ERR_INVALID_ARG;
+  const int64_t BT = Z->shape[0], V = Z->shape[1];
+  if (BT < 0 || V <= 0 || BT >= (1ll << 31) || V >= (1ll << 31)) return FLCE_ERR_INVALID_ARG;
+  if (BT > 0 && !check_matrix(Z, dt, BT, V)) return FLCE_ERR_INVALID_ARG;
+  if (target->dtype != FLCE_I64 || target->ndim != 1 || target->shape[0] != BT ||
+      (BT > 0 && (!target->data || target->stride[0] != 1)))
+    return FLCE_ERR_INVALID_ARG;
+  if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
+      (loss->ndim == 1 && loss->shape[0] != 1))
+    return FLCE_ERR_INVALID_ARG;
+  const int esz = dtype_size(dt);
+  if (BT > 0 && (!is_aligned(Z->data, 16) || (Z->stride[0] * esz) % 16)) return FLCE_ERR_INVALID_ARG;
+  if (grad && BT > 0) {
+    if (!check_matrix(grad, dt, BT, V)) return FLCE_ERR_INVALID_ARG;
+    if (!is_aligned(grad->data, 16) || (grad->stride[0] * esz) % 16) return FLCE_ERR_INVALID_ARG;
+  }
+  DeviceCtx* dev = nullptr;
+  flce_status st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+  if (BT == 0) return cudaMemsetAsync(loss->data, 0, 4, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  const int shift = 10;
+  const int64_t ntile = ceil_div(V, 1 << shift), ldp = round_up(BT, 32);
+  size_t o = 0;
+  const size_t off_nv = o; o = align256(o + 8);
+  const size_t off_rl = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_lse = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_zt = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_pm = o; o = align256(o + (size_t)ntile * ldp * 4);
+  const size_t off_ps = o; o = align256(o + (size_t)ntile * ldp * 4);
+  Workspace ws;
+  st = get_workspace(nullptr, o, stream, &ws);
+  if (st != FLCE_OK) return st;
+  uint8_t* b = static_cast<uint8_t*>(ws.ptr);
+  int64_t* nv_local = reinterpret_cast<int64_t*>(b + off_nv);
+  const int64_t* nv = (opt && opt->n_valid) ? opt->n_valid : nv_local;
+  float* rl = (opt && opt->row_loss) ? opt->row_loss : reinterpret_cast<float*>(b + off_rl);
+  float* lse = (opt && opt->lse) ? opt->lse : reinterpret_cast<float*>(b + off_lse);
+  float* zt = reinterpret_cast<float*>(b + off_zt);
+  float* pm = reinterpret_cast<float*>(b + off_pm);
+  float* ps = reinterpret_cast<float*>(b + off_ps);
+  const int64_t* tgt = static_cast<const int64_t*>(target->data);
+  Launcher L{stream, opt && (opt->flags & FLCE_FLAG_TIME_PHASES), env_debug() || (opt && (opt->flags & FLCE_FLAG_SYNC_CHECK))};
+  st = L.run(0, [&] { count_valid_kernel<<<1, 1024, 0, stream>>>(tgt, BT, V, ignore_index, nv_local, dev->err); });
+  if (st != FLCE_OK) return st;
+  const int64_t warps = BT * ntile;
+  if (dt == FLCE_BF16) {
+    CePartialArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data), Z->stride[0], tgt, ignore_index, V,
+                                   pm, ps, ldp, zt, (int)BT, (int)ntile, shift};
+    st = L.run(1, [&] { ce_partials_kernel<__nv_bfloat16><<<(unsigned)ceil_div(warps, 8), 256, 0, stream>>>(a); });
+  } else {
+    CePartialArgs<float> a{static_cast<const float*>(Z->data), Z->stride[0], tgt, ignore_index, V,
+                           pm, ps, ldp, zt, (int)BT, (int)ntile, shift};
+    st = L.run(1, [&] { ce_partials_kernel<float><<<(unsigned)ceil_div(warps, 8), 256, 0, stream>>>(a); });
+  }
+  if (st != FLCE_OK) return st;
+  for (int64_t r0 = 0; r0 < BT; r0 += 65535 * 32) {
+    const int rows = (int)std::min<int64_t>(65535 * 32, BT - r0);
+    CombineArgs a{tgt + r0, ignore_index, V, rows, (int)ntile, ldp, pm + r0, ps + r0, zt + r0, rl + r0, lse + r0, nv, reduction};
+    st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
+    if (st != FLCE_OK) return st;
+  }
+  if (grad) {
+    for (int64_t r0 = 0; r0 < BT; r0 += 65535) {
+      const int rows = (int)std::min<int64_t>(65535, BT - r0);
+      const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
+      if (dt == FLCE_BF16) {
+        CeGradArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
+                                    static_cast<__nv_bfloat16*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
+                                    tgt + r0, ignore_index, V, lse + r0, nv, reduction};
+        st = L.run(3, [&] { ce_grad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a); });
+      } else {
+        CeGradArgs<float> a{static_cast<const float*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
+                            static_cast<float*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
+                            tgt + r0, ignore_index, V, lse + r0, nv, reduction};
+        st = L.run(3, [&] { ce_grad_kernel<float><<<grid, 256, 0, stream>>>(a); });
+      }
+      if (st != FLCE_OK) return st;
+    }
+  }
+  return L.run(5, [&] {
+    finalize_loss_kernel<<<1, 1024, 0, stream>>>(rl, BT, nv, reduction, static_cast<float*>(loss->data));
+  });
+}
+
+}  // namespace
+}  // namespace flce
+
+using namespace flce;
+
+extern "C" {
+
+void flce_options_init(flce_options* opt) {
+  if (opt) std::memset(opt, 0, sizeof(*opt));
+}
+
+flce_status flce_fwd_bwd_ex(const flce_tensor* X, const flce_tensor* W, const flce_tensor* target,
+                            int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                            flce_tensor* grad_X, flce_tensor* grad_W, flce_stream_t stream,
+                            const flce_options* opt, flce_stats* stats) {
+  try {
+    return run_flce(X, W, target, ignore_index, reduction, loss, grad_X, grad_W,
+                    reinterpret_cast<cudaStream_t>(stream), opt, stats);
+  } catch (...) {
+    return FLCE_ERR_CUDA;
+  }
+}
+
+flce_status flce_fwd_bwd(const flce_tensor* X, const flce_tensor* W, const flce_tensor* target,
+                         int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                         flce_tensor* grad_X, flce_tensor* grad_W, flce_stream_t stream) {
+  return flce_fwd_bwd_ex(X, W, target, ignore_index, reduction, loss, grad_X, grad_W, stream,
+                         nullptr, nullptr);
+}
+
+flce_status flce_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, int32_t want_grad_W,
+                      const flce_options* opt, flce_stats* out) {
+  if (!out) return FLCE_ERR_INVALID_ARG;
+  Plan pl;
+  const flce_status st = make_plan(BT, H, V, dtype, want_grad_W != 0, opt, !(opt && opt->row_loss), &pl);
+  if (st != FLCE_OK) return st;
+  std::memset(out, 0, sizeof(*out));
+  out->chunk_rows = pl.chunk;
+  out->n_chunks = pl.n_chunks;
+  out->workspace_bytes = BT > 0 ? (int64_t)pl.total : 0;
+  out->materialized_logits_bytes = BT * V * 2;
+  out->path = dtype == FLCE_BF16 ? 1 : 0;
+  return FLCE_OK;
+}
+
+flce_status flce_count_valid(const flce_tensor* target, int64_t V, int64_t ignore_index,
+                             int64_t* n_valid_out, flce_stream_t stream) {
+  if (!target || !n_valid_out || V <= 0) return FLCE_ERR_INVALID_ARG;
+  if (target->dtype != FLCE_I64 || target->ndim != 1 || target->shape[0] < 0) return FLCE_ERR_INVALID_ARG;
+  const int64_t BT = target->shape[0];
+  if (BT > 0 && (!target->data || target->stride[0] != 1)) return FLCE_ERR_INVALID_ARG;
+  DeviceCtx* dev = nullptr;
+  const flce_status st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+  count_valid_kernel<<<1, 1024, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const int64_t*>(target->data), BT, V, ignore_index, n_valid_out, dev->err);
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+flce_status flce_cross_entropy(const flce_tensor* logits, const flce_tensor* target,
+                               int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                               flce_tensor* grad_logits, flce_stream_t stream,
+                               const flce_options* opt) {
+  try {
+    return run_ce(logits, target, ignore_index, reduction, loss, grad_logits,
+                  reinterpret_cast<cudaStream_t>(stream), opt);
+  } catch (...) {
+    return FLCE_ERR_CUDA;
+  }
+}
+
+flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N,
+                           int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn_major,
+                           int32_t b_mn_major, flce_stream_t stream) {
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0) return FLCE_ERR_INVALID_ARG;
+  if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return FLCE_ERR_INVALID_ARG;
+  if (lda % 8 || ldb % 8 || ldc % 4) return FLCE_ERR_INVALID_ARG;
+  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16)) return FLCE_ERR_INVALID_ARG;
+  if (lda < (a_mn_major ? M : K) || ldb < (b_mn_major ? N : K) || ldc < N) return FLCE_ERR_INVALID_ARG;
+  DeviceCtx* dev = nullptr;
+  const flce_status st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+  CUtensorMap ta, tb, z;
+  std::memset(&z, 0, sizeof(z));
+  const bool ok = (a_mn_major ? make_tmap(&ta, A, M, K, lda * 2, 64, 64) : make_tmap(&ta, A, K, M, lda * 2, 64, TC_BM)) &&
+                  (b_mn_major ? make_tmap(&tb, B, N, K, ldb * 2, 64, 64) : make_tmap(&tb, B, K, N, ldb * 2, 64, TC_BN));
+  if (!ok) return FLCE_ERR_CUDA;
+  TcParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.nprob = 1;
+  prm.prob[0] = make_problem((int)M, (int)N, (int)K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, EPI_STORE_F32, 1);
+  prm.prob[0].out = C;
+  prm.prob[0].ldo = ldc;
+  prm.err = dev->err;
+  launch_tc(ta, tb, z, z, prm, dev->sms, reinterpret_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (env_debug() && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
+
+flce_status flce_get_device_error(flce_stream_t stream, uint32_t* err) {
+  if (!err) return FLCE_ERR_INVALID_ARG;
+  DeviceCtx* dev = nullptr;
+  const flce_status st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaMemcpy(err, dev->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (cudaMemset(dev->err, 0, 4) != cudaSuccess) return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
+
+flce_status flce_phase_times(double* ms, int32_t* count, int32_t n_phases, int32_t reset) {
+  if (n_phases < 0) return FLCE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int p = 0; p < n_phases; ++p) {
+    if (ms) ms[p] = 0.0;
+    if (count) count[p] = 0;
+  }
+  for (const PhaseRec& r : g_phase_recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return FLCE_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (r.phase < n_phases) {
+      if (ms) ms[r.phase] += t;
+      if (count) count[r.phase] += 1;
+    }
+  }
+  if (reset) {
+    for (const PhaseRec& r : g_phase_recs) {
+      g_event_pool.push_back(r.a);
+      g_event_pool.push_back(r.b);
+    }
+    g_phase_recs.clear();
+  }
+  return FLCE_OK;
+}
+
+const char* flce_status_string(int32_t s) {
+  switch (s) {
+    case FLCE_OK: return "ok";
+    case FLCE_ERR_INVALID_ARG: return "invalid argument";
+    case FLCE_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case FLCE_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs sm_100)";
+    case FLCE_ERR_ALLOC: return "workspace allocation failed";
+    case FLCE_ERR_CUDA: return "CUDA error";
+    case FLCE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+int32_t flce_version(void) { return FLCE_VERSION; }
+
+}  // extern "C"

@@ -9,6 +9,7 @@ from .flce_oracle import (  # noqa: F401
     dlogits,
     flce,
     flce_brute_force,
+    flce_grad_W_rows,
     flce_rows,
     logits,
     row_logsumexp,

@@ -51,6 +51,7 @@ __all__ = [
     "dlogits",
     "flce",
     "flce_rows",
+    "flce_grad_W_rows",
     "flce_brute_force",
     "cross_entropy",
 ]
@@ -190,6 +191,22 @@ def flce_rows(X, W, target, rows: Sequence[int], n_valid: int,
     out = flce(_f64(X)[rows], W, np.asarray(target)[rows], ignore_index=ignore_index,
                reduction=reduction, n_valid=n_valid, want_grad_W=False)
     return {"row_loss": out["row_loss"], "lse": out["lse"], "grad_X": out["grad_X"]}
+
+
+def flce_grad_W_rows(X, W, target, vocab_rows: Sequence[int], ignore_index: int = -100,
+                     reduction: str = "mean", n_valid: Optional[int] = None) -> np.ndarray:
+    """grad_W[v, :] = sum_i dz[i, v] X_i for the listed vocabulary rows only.
+
+    Every row's lse still needs all V logits; only the final contraction is
+    restricted to the requested rows of grad_W.
+    """
+    X = _f64(X)
+    target = np.asarray(target, dtype=np.int64)
+    z = logits(X, W)
+    valid = valid_mask(target, z.shape[1], ignore_index)
+    N = int(valid.sum()) if n_valid is None else int(n_valid)
+    dz = _softmax_minus_onehot(z, row_logsumexp(z), target, valid, _scale(reduction, N))
+    return _grad_W(dz[:, np.asarray(vocab_rows, dtype=np.int64)], X)
 
 
 def flce_brute_force(X, W, target, ignore_index: int = -100,

@@ -1,0 +1,160 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_cross_entropy_04_b200 import _binding as B
+from linear_cross_entropy_04_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flce.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FLCE_API\s+[\w\s\*]+?\b(flce_\w+)\s*\(", text)))
+
+
+def exported_symbols():
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    return {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+
+
+def test_every_declared_entry_point_is_exported(lib):
+    decl = declared_functions()
+    assert len(decl) >= 11
+    exported = exported_symbols()
+    missing = [d for d in decl if d not in exported]
+    assert not missing, missing
+    for d in decl:
+        assert hasattr(lib, d)
+
+
+def test_binding_signatures_cover_the_header():
+    assert set(declared_functions()) == set(B._SIGS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.flce_version() == 100
+    assert lib.flce_status_string(0) == b"ok"
+    assert b"unsupported device" in lib.flce_status_string(3)
+    assert lib.flce_status_string(99) == b"unknown status"
+
+
+def _t(ptr, dtype, shape, stride=None):
+    d = B.FlceTensor()
+    d.data = ptr
+    d.dtype = dtype
+    d.ndim = len(shape)
+    for i, n in enumerate(shape):
+        d.shape[i] = n
+    if stride is None:
+        stride = [1] * len(shape)
+        for i in range(len(shape) - 2, -1, -1):
+            stride[i] = stride[i + 1] * shape[i + 1]
+    for i, s in enumerate(stride):
+        d.stride[i] = s
+    return d
+
+
+FAKE = 0x10000  # never dereferenced: validation fails before any device work
+
+
+def _call(lib, X, W, tg, loss, gX=None, gW=None, reduction=0):
+    ref = lambda t: ctypes.byref(t) if t is not None else None  # noqa: E731
+    return lib.flce_fwd_bwd(ref(X), ref(W), ref(tg), -100, reduction, ref(loss), ref(gX), ref(gW), None)
+
+
+@pytest.mark.parametrize("case", ["null_X", "null_loss", "dtype_mix", "bad_dtype", "shape_H", "target_len",
+                                  "target_dtype", "stride", "bad_reduction", "bf16_H_mod8", "bf16_misaligned",
+                                  "grad_shape", "loss_shape"])
+def test_invalid_arguments_are_rejected_on_the_host(lib, case):
+    X = _t(FAKE, B.BF16, (64, 128))
+    W = _t(FAKE, B.BF16, (1000, 128))
+    tg = _t(FAKE, B.I64, (64,))
+    loss = _t(FAKE, B.F32, ())
+    gX, gW, red = None, None, 0
+    expect = 1
+    if case == "null_X":
+        X = None
+    elif case == "null_loss":
+        loss = None
+    elif case == "dtype_mix":
+        W = _t(FAKE, B.F32, (1000, 128))
+        expect = 2
+    elif case == "bad_dtype":
+        X = _t(FAKE, B.I64, (64, 128))
+        expect = 2
+    elif case == "shape_H":
+        W = _t(FAKE, B.BF16, (1000, 120))
+    elif case == "target_len":
+        tg = _t(FAKE, B.I64, (63,))
+    elif case == "target_dtype":
+        tg = _t(FAKE, B.F32, (64,))
+    elif case == "stride":
+        X = _t(FAKE, B.BF16, (64, 128), stride=(128, 2))
+    elif case == "bad_reduction":
+        red = 7
+    elif case == "bf16_H_mod8":
+        X = _t(FAKE, B.BF16, (64, 100))
+        W = _t(FAKE, B.BF16, (1000, 100))
+    elif case == "bf16_misaligned":
+        X = _t(FAKE + 2, B.BF16, (64, 128))
+    elif case == "grad_shape":
+        gW = _t(FAKE, B.BF16, (999, 128))
+    elif case == "loss_shape":
+        loss = _t(FAKE, B.F32, (2,))
+    assert _call(lib, X, W, tg, loss, gX, gW, red) == expect
+
+
+def test_other_entry_points_validate(lib):
+    assert lib.flce_gemm_bf16(None, None, None, 1, 1, 1, 8, 8, 4, 0, 0, None) == 1
+    assert lib.flce_gemm_bf16(FAKE, FAKE, FAKE, 16, 16, 16, 12, 16, 16, 0, 0, None) == 1  # lda % 8
+    assert lib.flce_count_valid(None, 10, -100, None, None) == 1
+    z = _t(FAKE, B.BF16, (4, 100))
+    tg = _t(FAKE, B.I64, (3,))
+    loss = _t(FAKE, B.F32, ())
+    assert lib.flce_cross_entropy(ctypes.byref(z), ctypes.byref(tg), -100, 0, ctypes.byref(loss), None, None,
+                                  None) == 1
+    assert lib.flce_get_device_error(None, None) == 1
+    assert lib.flce_phase_times(None, None, -1, 0) == 1
+
+
+def test_plan_is_host_only_and_bounded(lib):
+    from linear_cross_entropy_04_b200.inputs import WORKLOADS
+    from linear_cross_entropy_04_b200 import plan
+
+    for w in WORKLOADS.values():
+        p = plan(w.BT, w.H, w.V, w.dtype)
+        assert p["n_chunks"] >= 2, w.name  # the logits of the whole batch are never held
+        assert p["chunk_rows"] % 128 == 0 and p["chunk_rows"] * (p["n_chunks"] - 1) < w.BT
+        if w.dtype == "bf16":
+            assert p["workspace_bytes"] <= (512 << 20) + (64 << 20)
+            assert p["workspace_bytes"] < 0.55 * w.BT * w.V * 2
+    p = plan(4096, 4096, 128256, chunk_rows=1000)
+    assert p["chunk_rows"] == 1024 and p["n_chunks"] == 4
+    p = plan(4096, 4096, 128256, workspace_limit_bytes=300 << 20)
+    assert p["workspace_bytes"] <= (300 << 20) + (8 << 20)
+    acc = plan(4096, 4096, 128256, grad_w_accum="fp32")
+    assert acc["workspace_bytes"] - plan(4096, 4096, 128256)["workspace_bytes"] >= 128256 * 4096 * 4
+    st = B.FlceStats()
+    assert lib.flce_plan(10, 0, 10, B.BF16, 1, None, ctypes.byref(st)) == 1
+    assert lib.flce_plan(10, 8, 10, B.I64, 1, None, ctypes.byref(st)) == 2
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", "/nonexistent/libflce.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        B.lib()

@@ -1,0 +1,217 @@
+"""CUDA path vs the float64 oracle, element by element, at sizes the oracle
+finishes in seconds (several tiles, ragged tails), plus the edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_cross_entropy_04_b200.inputs import WORKLOADS, make_inputs, IGNORE_INDEX
+from flce_testlib import need_gpu, to_dev, rel_err, assert_grad_close, TOL
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def L():
+    import linear_cross_entropy_04_b200 as lib
+
+    return lib
+
+
+def run_case(d, reduction="mean", chunk_rows=0, grad_w_accum="output", ignore_index=IGNORE_INDEX,
+             want_grad_X=True, want_grad_W=True):
+    X, W, t = to_dev(d)
+    row_loss = torch.empty(d["BT"], dtype=torch.float32, device="cuda")
+    loss, gX, gW, st = L().fused_linear_cross_entropy(
+        X, W, t, ignore_index=ignore_index, reduction=reduction, chunk_rows=chunk_rows,
+        grad_w_accum=grad_w_accum, row_loss=row_loss, want_grad_X=want_grad_X, want_grad_W=want_grad_W,
+        return_stats=True)
+    torch.cuda.synchronize()
+    assert L().device_error() == 0
+    ref = oracle.flce(d["X"], d["W"], d["target"], ignore_index=ignore_index, reduction=reduction)
+    tol = TOL[d["dtype"]]
+    assert rel_err(loss.item(), ref["loss"]) <= tol["loss"], (loss.item(), ref["loss"])
+    np.testing.assert_allclose(row_loss.cpu().numpy(), ref["row_loss"], rtol=tol["loss"], atol=tol["loss"])
+    if want_grad_X:
+        assert_grad_close(gX, ref["grad_X"], d["dtype"], "grad_X")
+        ign = d["target"] == ignore_index
+        if ign.any():
+            assert torch.all(gX[torch.from_numpy(ign).cuda()] == 0), "ignored rows must get exactly 0"
+    if want_grad_W:
+        assert_grad_close(gW, ref["grad_W"], d["dtype"], "grad_W")
+    return st
+
+
+# ------------------------------------------------------------ tcgen05 engine alone
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 520, 200), (1024, 768, 2048), (129, 8, 4099)])
+def test_engine_gemm_matches_torch(a_mn, b_mn, M, N, K):
+    g = torch.Generator().manual_seed(M * 7 + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    Bm = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    ref = A.float() @ Bm.float().T
+    # the engine wants leading dimensions that are multiples of 8 elements
+    def lay(T, mn):
+        S = T.T.contiguous() if mn else T.contiguous()
+        cols = S.shape[1]
+        pad = (-cols) % 8
+        return torch.nn.functional.pad(S, (0, pad)).cuda()[:, :cols]
+    Ad, Bd = lay(A, a_mn), lay(Bm, b_mn)
+    C = L().gemm_bf16(Ad, Bd, M, N, K, bool(a_mn), bool(b_mn))
+    torch.cuda.synchronize()
+    assert L().device_error() == 0
+    err = (C.cpu() - ref).abs().max().item()
+    assert err <= 1e-3 * ref.abs().max().item() + 1e-3, err
+
+
+# ------------------------------------------------------------ FLCE parity
+
+def test_tiny_fp32_config():
+    d = make_inputs(WORKLOADS["tiny"])
+    st = run_case(d)
+    assert st["path"] == 0 and st["n_chunks"] >= 2
+
+
+@pytest.mark.parametrize("reduction", ["mean", "sum"])
+def test_tiny_fp32_sum_and_chunks(reduction):
+    d = make_inputs(WORKLOADS["tiny"], BT=300, V=1000)
+    run_case(d, reduction=reduction, chunk_rows=128)
+
+
+@pytest.mark.parametrize("BT,H,V", [(512, 256, 4096), (300, 192, 1000), (129, 192, 4099), (1000, 512, 3000),
+                                    (64, 8, 300)])
+def test_bf16_small_shapes(BT, H, V):
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=BT, H=H, V=V)
+    run_case(d)
+
+
+@pytest.mark.parametrize("accum", ["output", "fp32"])
+def test_bf16_many_chunks_ragged(accum):
+    d = make_inputs(WORKLOADS["qwen2_7b"], BT=700, H=256, V=2000)
+    st = run_case(d, chunk_rows=256, grad_w_accum=accum)
+    assert st["n_chunks"] == 3
+
+
+def test_bf16_sum_reduction_and_wide_logits():
+    d = make_inputs(WORKLOADS["large_vocab_stress"], BT=400, H=512, V=5000)
+    run_case(d, reduction="sum")
+
+
+def test_bf16_ignore_index_inside_vocab():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=200, H=64, V=700)
+    ii = int(d["target"][d["target"] >= 0][0])
+    d["target"][d["target"] == IGNORE_INDEX] = ii  # -100 would now be out of range
+    run_case(d, ignore_index=ii)
+
+
+def test_bf16_only_one_gradient():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=300, H=128, V=900)
+    run_case(d, want_grad_X=False)
+    run_case(d, want_grad_W=False)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_all_rows_ignored(dtype):
+    w = WORKLOADS["tiny"] if dtype == "f32" else WORKLOADS["llama3_8b_seq"]
+    d = make_inputs(w, BT=150, H=64, V=500)
+    d["target"][:] = IGNORE_INDEX
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t)
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0
+    assert torch.all(gX == 0) and torch.all(gW == 0)
+
+
+def test_empty_batch_zeroes_grad_W():
+    W = torch.randn(300, 64, device="cuda").to(torch.bfloat16)
+    X = torch.empty(0, 64, device="cuda", dtype=torch.bfloat16)
+    t = torch.empty(0, dtype=torch.int64, device="cuda")
+    gW = torch.full_like(W, 7.0)
+    loss = torch.full((), 3.0, device="cuda")
+    L().fused_linear_cross_entropy(X, W, t, out=(loss, None, gW))
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0 and torch.all(gW == 0)
+
+
+def test_w_zero_closed_form_bf16():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=500, H=256, V=3000, w_zero=True)
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t)
+    torch.cuda.synchronize()
+    assert rel_err(loss.item(), np.log(3000)) <= 1e-3
+    assert torch.all(gX == 0)
+    ref = oracle.flce(d["X"], d["W"], d["target"])["grad_W"]
+    assert_grad_close(gW, ref, "bf16", "grad_W (W=0)")
+
+
+def test_out_of_range_target_sets_the_error_word():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=64, H=64, V=300)
+    d["target"][5] = 300
+    X, W, t = to_dev(d)
+    L().fused_linear_cross_entropy(X, W, t)
+    assert L().device_error() & 0x1
+    assert L().device_error() == 0  # reading clears it
+
+
+def test_deterministic():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=600, H=256, V=3000)
+    X, W, t = to_dev(d)
+    a = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256)
+    b = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256)
+    torch.cuda.synchronize()
+    assert a[0].item() == b[0].item()
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_cross_entropy_logits_given(dtype, inplace):
+    rng = np.random.default_rng(4)
+    BT, V = 300, 5003
+    z = (rng.standard_normal((BT, V)) * 3).astype(np.float32)
+    t = rng.integers(0, V, BT)
+    t[::7] = IGNORE_INDEX
+    zt = torch.from_numpy(z).to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+    z64 = zt.double().numpy()
+    ref = oracle.cross_entropy(z64, t)
+    # rows of 5003 elements are not 16-byte aligned: pad the row pitch
+    pitch = 5008
+    buf = torch.zeros(BT, pitch, dtype=zt.dtype)
+    buf[:, :V] = zt
+    zd = buf.cuda()[:, :V]
+    loss, g = L().cross_entropy(zd, torch.from_numpy(t).cuda(), inplace=inplace)
+    torch.cuda.synchronize()
+    assert rel_err(loss.item(), ref["loss"]) <= TOL[dtype]["loss"]
+    assert_grad_close(g, ref["dz"], dtype, "dz")
+    if inplace:
+        assert g.data_ptr() == zd.data_ptr()
+
+
+def test_module_autograd_matches_oracle():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
+    X, W, t = to_dev(d)
+    X = X.reshape(2, 128, 128).clone().requires_grad_(True)
+    W = W.clone().requires_grad_(True)
+    loss = L().FusedLinearCrossEntropyLoss()(W, X, t.reshape(2, 128))
+    (2.5 * loss).backward()
+    ref = oracle.flce(d["X"], d["W"], d["target"])
+    assert rel_err(loss.item(), ref["loss"]) <= 1e-3
+    assert_grad_close(X.grad.reshape(256, 128), 2.5 * ref["grad_X"], "bf16", "module grad_X")
+    assert_grad_close(W.grad, 2.5 * ref["grad_W"], "bf16", "module grad_W")
+
+
+def test_host_buffers_end_to_end():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
+    X = torch.from_numpy(d["X"]).to(torch.bfloat16).pin_memory()
+    W = torch.from_numpy(d["W"]).to(torch.bfloat16).pin_memory()
+    t = torch.from_numpy(d["target"]).pin_memory()
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t)
+    assert not loss.is_cuda and not gW.is_cuda
+    ref = oracle.flce(d["X"], d["W"], d["target"])
+    assert rel_err(loss.item(), ref["loss"]) <= 1e-3
+    assert_grad_close(gW, ref["grad_W"], "bf16", "grad_W")

@@ -266,6 +266,16 @@ def test_flce_rows_matches_full_batch():
     np.testing.assert_allclose(r["grad_X"], full["grad_X"][rows], atol=1e-15)
 
 
+def test_flce_grad_W_rows_matches_full():
+    X, W, t = _rand_case(BT=25, H=4, V=19, ignore=(3,))
+    full = oracle.flce(X, W, t)
+    for red in ("mean", "sum"):
+        full = oracle.flce(X, W, t, reduction=red)
+        vr = np.array([0, 4, 18, int(t[0])])
+        np.testing.assert_allclose(oracle.flce_grad_W_rows(X, W, t, vr, reduction=red),
+                                   full["grad_W"][vr], atol=1e-15)
+
+
 def test_cross_entropy_matches_torch_and_flce():
     X, W, t = _rand_case(BT=9, H=4, V=15, ignore=(0,))
     z = oracle.logits(X, W)
