@@ -1,0 +1,368 @@
+"""Benchmark: fused linear cross-entropy forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one full pass of the path (count, logits GEMM + online softmax,
+row combine, in-place dlogits, grad_X/grad_W GEMMs, loss) over one batch of
+synthetic tokens of the named workload (default: Llama-3-8B lm_head, BT=4096,
+H=4096, V=128256, bf16). Inputs stay resident in HBM; W alone (1.05 GB) is
+larger than the 126 MB L2, so no L2 flush is needed between steps.
+
+With N > 1 (torchrun), every rank runs its own batch (weak scaling) with a
+replica of W, and the step adds the data-parallel exchange: an all-reduce of
+the non-ignored row count before the loss, then of the loss and of grad_W.
+
+--impl reference times the float64 CPU oracle on bounded samples of the same
+workload (rank 0 only); it is the slow baseline the pages' method is exact to.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FLCE fwd+bwd tokens/sec and TFLOP/s (% of B200 bf16 peak), peak workspace"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama3_8b_seq")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--chunk-rows", type=int, default=0)
+    ap.add_argument("--grad-w-accum", default="output", choices=["output", "fp32"])
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s in sm if mx and s > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(d, n_rows, Wf64=None):
+    """Run the float64 oracle on the first n_rows tokens: the full per-token work
+    (logits over V, loss, grad_X rows, their grad_W contribution). Returns seconds."""
+    import numpy as np
+    import oracle
+
+    n_valid = oracle.count_valid(d["target"], d["V"])
+    X = d["X"][:n_rows].astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.flce(X, Wf64, d["target"][:n_rows], n_valid=n_valid)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:  # noqa: BLE001
+        return os.cpu_count()
+
+
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(d, target_s):
+    import numpy as np
+
+    Wf = d["W"].astype(np.float64)
+    t = oracle_sample(d, 8, Wf)
+    rows = int(max(8, min(2048, 8 * target_s / max(t, 1e-3))))
+    t = oracle_sample(d, rows, Wf)
+    return {"value": rows / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {rows} tokens of the workload, full fwd+bwd per token in float64 NumPy "
+                      f"({t:.1f} s), on {cpu_model()}",
+            "seconds": t}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    from linear_cross_entropy_04_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    d = make_inputs(w)
+    Wf = d["W"].astype(np.float64)
+    t1 = oracle_sample(d, 4, Wf)
+    rows = int(max(4, min(1024, 4 * (150.0 / max(1, args.steps + args.warmup)) / max(t1, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(d, rows, Wf)
+    tot = 0.0
+    for _ in range(args.steps):
+        tot += oracle_sample(d, rows, Wf)
+    value = rows * args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "BT": w.BT, "H": w.H, "V": w.V,
+                                            "sample_tokens_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"each step: the first {rows} tokens, full fwd+bwd in float64 NumPy, "
+                                       f"on {cpu_model()}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import linear_cross_entropy_04_b200 as flce
+    from linear_cross_entropy_04_b200 import _binding as B
+    from linear_cross_entropy_04_b200.inputs import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = WORKLOADS[args.workload]
+    d = make_inputs(w, seed=w.seed + rank)
+    dev = torch.device("cuda", local)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    X = torch.from_numpy(d["X"]).to(dt).to(dev)
+    W = torch.from_numpy(d["W"]).to(dt).to(dev)
+    t = torch.from_numpy(d["target"]).to(dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    gX = torch.empty_like(X)
+    gW = torch.empty_like(W)
+    nvalid = torch.empty((), dtype=torch.int64, device=dev)
+    kw = dict(chunk_rows=args.chunk_rows, grad_w_accum=args.grad_w_accum)
+
+    def step(flags=0):
+        nv = None
+        if world > 1:
+            nv = flce.count_valid(t, w.V)
+            dist.all_reduce(nv)
+        _, _, _, st = flce.fused_linear_cross_entropy(X, W, t, out=(loss, gX, gW), n_valid=nv, flags=flags,
+                                                      return_stats=True, **kw)
+        if world > 1:
+            dist.all_reduce(loss)
+            dist.all_reduce(gW)
+        return st
+
+    mem0 = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    for _ in range(args.warmup):
+        st = step()
+    torch.cuda.synchronize()
+    if flce.device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    peak_extra_torch = torch.cuda.max_memory_allocated(dev) - mem0
+    flce.phase_times(reset=True)
+
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            st = step(flags=B.FLAG_TIME_PHASES)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        mt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(mt, op=dist.ReduceOp.MAX)
+        ms = float(mt.item())
+    phases = flce.phase_times(reset=True)
+    err = flce.device_error()
+
+    ms_step = ms / args.steps
+    tokens = w.BT * world * args.steps
+    value = tokens / (ms / 1e3)
+    tflops = w.useful_flops * world * args.steps / (ms / 1e3) / 1e12
+    peaks = load_peaks()
+
+    # roofline of the dominant kernel (its own CUDA-event time inside the timed region)
+    flops_per_phase = {"logits_gemm_softmax": 2.0 * w.BT * w.H * w.V * args.steps,
+                       "grad_gemms": 4.0 * w.BT * w.H * w.V * args.steps}
+    dom = max(phases, key=lambda k: phases[k][0])
+    dom_ms, dom_n = phases[dom]
+    if dom in flops_per_phase:
+        achieved = flops_per_phase[dom] / (dom_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_kind": f"{peaks['source']} sustained bf16 (kernel runs inside a long step loop)",
+                "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                "launches": dom_n, "avg_launch_ms": dom_ms / max(dom_n, 1)}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": None}
+    gemm_ms = sum(phases[k][0] for k in flops_per_phase)
+    all_ms = sum(v[0] for v in phases.values())
+
+    # end to end through the public API with host buffers: inputs H2D, results D2H
+    e2e = None
+    if world == 1 and args.e2e_steps > 0:
+        Xh = X.cpu().pin_memory()
+        Wh = W.cpu().pin_memory()
+        th = t.cpu().pin_memory()
+        hout = (torch.empty((), dtype=torch.float32).pin_memory(), torch.empty_like(Xh).pin_memory(),
+                torch.empty_like(Wh).pin_memory())
+        kw["host_out"] = hout
+        for _ in range(1):
+            flce.fused_linear_cross_entropy(Xh, Wh, th, **kw)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            lh, gxh, gwh = flce.fused_linear_cross_entropy(Xh, Wh, th, **kw)
+        e1.record()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        e_ms = max(e0.elapsed_time(e1), wall * 1e3)
+        h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size() + th.numel() * 8
+        d2h = 4 + gxh.numel() * gxh.element_size() + gwh.numel() * gwh.element_size()
+        e2e = {"value": w.BT * args.e2e_steps / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.e2e_steps,
+               "how": "public API with pinned host X, W, target; loss, grad_X, grad_W copied back to pinned "
+                      "host buffers each step"}
+        del Xh, Wh, th, hout
+        kw.pop("host_out")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(d, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; random-init lm_head weights)",
+        "config": {"workload": w.name, "BT": w.BT, "H": w.H, "V": w.V, "global_batch": w.BT * world,
+                   "seq_len": w.BT, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (W alone is %.2f GB)" % (w.V * w.H * 2 / 1e9),
+                   "chunk_rows": st["chunk_rows"], "n_chunks": st["n_chunks"],
+                   "grad_w_accum": args.grad_w_accum},
+        "tflops": tflops,
+        "frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"],
+        "frac_of_bf16_burst_peak": tflops / peaks["bf16_tflops"],
+        "peak_workspace_bytes": st["workspace_bytes"],
+        "peak_extra_torch_bytes": peak_extra_torch,
+        "materialized_logits_bytes": st["materialized_logits_bytes"],
+        "workspace_vs_materialized": st["workspace_bytes"] / st["materialized_logits_bytes"],
+        "phases_ms_per_step": {k: v[0] / args.steps for k, v in phases.items()},
+        "gemm_share_of_step": gemm_ms / max(all_ms, 1e-9),
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": st["kernel_launches"] * args.steps,
+        "clocks": clk.summary(),
+        "device_error": err,
+        "peaks": peaks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

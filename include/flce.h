@@ -57,7 +57,7 @@ typedef enum {
   FLCE_ERR_INVALID_ARG = 1,        /* null pointer, bad shape, stride or alignment */
   FLCE_ERR_UNSUPPORTED_DTYPE = 2,  /* dtype combination not provided */
   FLCE_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not sm_100 (B200); caller may fall back */
-  FLCE_ERR_ALLOC = 4,              /* stream-ordered workspace allocation failed */
+  FLCE_ERR_ALLOC = 4,              /* workspace allocation from the library's pool failed */
   FLCE_ERR_CUDA = 5,               /* a CUDA runtime call failed */
   FLCE_ERR_WORKSPACE_TOO_SMALL = 6 /* caller-provided workspace smaller than the plan needs */
 } flce_status;
@@ -126,7 +126,9 @@ FLCE_API void flce_options_init(flce_options* opt);
  *   grad_W  [V,H]   same dtype as W, or NULL to skip: fully overwritten
  * bf16 runs the tcgen05 tensor-core path (fp32 accumulation, bf16 results,
  * H % 8 == 0, 16-byte aligned rows); f32 runs an exact-fp32 SIMT path.
- * Workspace is taken stream-ordered (cudaMallocAsync) and released at the end.
+ * Unless opt->workspace is given, workspace is taken stream-ordered from a
+ * library-owned memory pool (cudaMallocFromPoolAsync) and released to it at
+ * the end; the pool keeps the memory mapped for the next call.
  */
 FLCE_API flce_status flce_fwd_bwd(const flce_tensor* X, const flce_tensor* W, const flce_tensor* target,
                          int64_t ignore_index, int32_t reduction, flce_tensor* loss,

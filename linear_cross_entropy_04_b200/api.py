@@ -41,13 +41,16 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                chunk_rows: int = 0, workspace_limit_bytes: int = 0,
                                grad_w_accum: str = "output", n_valid: Optional[torch.Tensor] = None,
                                row_loss: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                               flags: int = 0, stream=None, out=None, return_stats: bool = False):
+                               flags: int = 0, stream=None, out=None, host_out=None,
+                               return_stats: bool = False):
     """Loss, grad_X and grad_W of cross-entropy over X W^T in one call.
 
     X [BT, H] and W [V, H] (bf16 or fp32, CUDA), target [BT] int64.
     Tensors on the host are staged to the current CUDA device and the
     results copied back (the end-to-end path); nothing runs on the CPU.
+    host_out = (loss, grad_X, grad_W) pinned host tensors receive them then.
     out = (loss, grad_X, grad_W) preallocated device tensors may be given.
+    The library's workspace is taken from torch's caching allocator.
     Returns (loss [scalar fp32], grad_X or None, grad_W or None[, stats]).
     """
     host = not X.is_cuda
@@ -64,6 +67,13 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
         gW = torch.empty_like(W) if want_grad_W else None
     o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags, n_valid, row_loss, lse)
     st = B.FlceStats()
+    B.check(B.lib().flce_plan(X.shape[0], X.shape[1], W.shape[0], B.dtype_code(X), int(gW is not None),
+                              ctypes.byref(o), ctypes.byref(st)), "flce_plan")
+    ws = None
+    if st.workspace_bytes > 0:
+        ws = torch.empty(st.workspace_bytes, dtype=torch.uint8, device=X.device)
+        o.workspace = ws.data_ptr()
+        o.workspace_bytes = st.workspace_bytes
     tX, tW, tt, tl = B.tensor(X), B.tensor(W), B.tensor(target), B.tensor(loss)
     tgX = B.tensor(gX) if gX is not None else None
     tgW = B.tensor(gW) if gW is not None else None
@@ -74,9 +84,19 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                  B.stream_handle(stream), ctypes.byref(o), ctypes.byref(st))
     B.check(rc, "flce_fwd_bwd_ex")
     if host:
-        loss = loss.to("cpu", non_blocking=False)
-        gX = gX.cpu() if gX is not None else None
-        gW = gW.cpu() if gW is not None else None
+        if host_out is not None:
+            hl, hx, hw = host_out
+            hl.copy_(loss, non_blocking=True)
+            if gX is not None:
+                hx.copy_(gX, non_blocking=True)
+            if gW is not None:
+                hw.copy_(gW, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+            loss, gX, gW = hl, (hx if gX is not None else None), (hw if gW is not None else None)
+        else:
+            loss = loss.to("cpu", non_blocking=False)
+            gX = gX.cpu() if gX is not None else None
+            gW = gW.cpu() if gW is not None else None
     res = (loss, gX, gW)
     return res + (st.as_dict(),) if return_stats else res
 

@@ -40,6 +40,7 @@ struct DeviceCtx {
   bool supported = false;
   int sms = 0;
   uint32_t* err = nullptr;
+  cudaMemPool_t pool = nullptr;  // library-owned stream-ordered pool for workspaces
 };
 
 std::mutex g_mu;
@@ -73,6 +74,18 @@ flce_status device_ctx(DeviceCtx** out) {
         return FLCE_ERR_CUDA;
       if (cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TC_SMEM_BYTES) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+      // A private pool that keeps freed workspace mapped, so repeated calls
+      // reuse it stream-ordered instead of mapping and unmapping memory.
+      cudaMemPoolProps pp;
+      std::memset(&pp, 0, sizeof(pp));
+      pp.allocType = cudaMemAllocationTypePinned;
+      pp.handleTypes = cudaMemHandleTypeNone;
+      pp.location.type = cudaMemLocationTypeDevice;
+      pp.location.id = dev;
+      if (cudaMemPoolCreate(&c.pool, &pp) != cudaSuccess) return FLCE_ERR_CUDA;
+      uint64_t keep = ~0ull;
+      if (cudaMemPoolSetAttribute(c.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
         return FLCE_ERR_CUDA;
       if (!g_encode) {
         void* fn = nullptr;
@@ -231,7 +244,7 @@ struct Workspace {
 };
 
 flce_status get_workspace(const flce_options* opt, size_t bytes, cudaStream_t stream,
-                          Workspace* ws) {
+                          cudaMemPool_t pool, Workspace* ws) {
   ws->stream = stream;
   if (opt && opt->workspace) {
     if ((size_t)opt->workspace_bytes < bytes) return FLCE_ERR_WORKSPACE_TOO_SMALL;
@@ -239,7 +252,7 @@ flce_status get_workspace(const flce_options* opt, size_t bytes, cudaStream_t st
     ws->ptr = opt->workspace;
     return FLCE_OK;
   }
-  if (cudaMallocAsync(&ws->ptr, bytes, stream) != cudaSuccess) {
+  if (cudaMallocFromPoolAsync(&ws->ptr, bytes, pool, stream) != cudaSuccess) {
     cudaGetLastError();
     ws->ptr = nullptr;
     return FLCE_ERR_ALLOC;
@@ -335,7 +348,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   }
 
   Workspace ws;
-  st = get_workspace(opt, pl.total, stream, &ws);
+  st = get_workspace(opt, pl.total, stream, dev->pool, &ws);
   if (st != FLCE_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(ws.ptr);
   int64_t* nvalid_local = reinterpret_cast<int64_t*>(base + pl.off_nvalid);
@@ -533,7 +546,7 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   const size_t off_pm = o; o = align256(o + (size_t)ntile * ldp * 4);
   const size_t off_ps = o; o = align256(o + (size_t)ntile * ldp * 4);
   Workspace ws;
-  st = get_workspace(nullptr, o, stream, &ws);
+  st = get_workspace(nullptr, o, stream, dev->pool, &ws);
   if (st != FLCE_OK) return st;
   uint8_t* b = static_cast<uint8_t*>(ws.ptr);
   int64_t* nv_local = reinterpret_cast<int64_t*>(b + off_nv);
