@@ -13,7 +13,8 @@ import os
 import threading
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libflce.so")
+# FLCE_LIBRARY may name another build of the same library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("FLCE_LIBRARY") or os.path.join(PKG, "libflce.so")
 
 F32, BF16, I64 = 0, 1, 2
 MEAN, SUM = 0, 1

@@ -27,10 +27,11 @@ def nvcc_path():
     raise RuntimeError("nvcc not found")
 
 
-def command(verbose=False):
+def command(verbose=False, out=OUT, defines=()):
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
            "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared",
-           "-cudart", "static", "-I", os.path.join(ROOT, "include"), "-o", OUT, SRC]
+           "-cudart", "static", "-I", os.path.join(ROOT, "include"), "-o", out, SRC]
+    cmd[1:1] = [f"-D{d}" for d in defines]
     if verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     return cmd
@@ -43,15 +44,16 @@ def up_to_date():
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force=False, verbose=False):
-    if not force and up_to_date():
+def build(force=False, verbose=False, out=None, defines=()):
+    """Compile the library; out/defines build a variant (e.g. tuning knobs) elsewhere."""
+    if out is None and not force and up_to_date():
         return OUT
-    r = subprocess.run(command(verbose), capture_output=True, text=True)
+    r = subprocess.run(command(verbose, out or OUT, defines), capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    return OUT
+    return out or OUT
 
 
 if __name__ == "__main__":

@@ -24,6 +24,7 @@
 #include "../../include/flce.h"
 #include "aux_kernels.cuh"
 #include "tc_gemm.cuh"
+#include "tc_gemm2.cuh"
 
 namespace flce {
 
@@ -39,6 +40,7 @@ struct DeviceCtx {
   bool init = false;
   bool supported = false;
   int sms = 0;
+  int pairs = 0;  // CTA pairs of the cluster engine that fit on the device at once
   uint32_t* err = nullptr;
   cudaMemPool_t pool = nullptr;  // library-owned stream-ordered pool for workspaces
 };
@@ -73,8 +75,30 @@ flce_status device_ctx(DeviceCtx** out) {
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.err), g_err_word) != cudaSuccess)
         return FLCE_ERR_CUDA;
       if (cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               TC_SMEM_BYTES) != cudaSuccess)
+                               TC_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tc_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               T2_SMEM_BYTES) != cudaSuccess)
         return FLCE_ERR_CUDA;
+      {
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (c.sms / 2));
+        cfg.blockDim = dim3(TC_THREADS);
+        cfg.dynamicSmemBytes = T2_SMEM_BYTES;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int nc = 0;
+        if (cudaOccupancyMaxActiveClusters(&nc, tc_gemm_pair_kernel, &cfg) != cudaSuccess || nc <= 0) {
+          cudaGetLastError();
+          nc = c.sms / 2;
+        }
+        c.pairs = std::min(nc, c.sms / 2);
+      }
       // A private pool that keeps freed workspace mapped, so repeated calls
       // reuse it stream-ordered instead of mapping and unmapping memory.
       cudaMemPoolProps pp;
@@ -261,13 +285,34 @@ flce_status get_workspace(const flce_options* opt, size_t bytes, cudaStream_t st
   return FLCE_OK;
 }
 
-TcProblem make_problem(int M, int N, int K, int a_mn, int b_mn, int epi, int m_fastest) {
+// Tensor-core engine: the CTA-pair kernel (256 x 256 tiles, default) or the
+// single-CTA kernel (128 x 256 tiles), chosen with FLCE_ENGINE=2sm|1sm.
+struct Engine {
+  bool pair;
+  int bm;         // tile rows
+  int b_box_rows; // rows of B in one K-major TMA box (per CTA)
+};
+
+Engine engine() {
+  const char* s = std::getenv("FLCE_ENGINE");
+  if (s && std::strcmp(s, "1sm") == 0) return Engine{false, TC_BM, TC_BN};
+  return Engine{true, T2_BM, T2_HALF};
+}
+
+// grad_X and grad_W of a chunk in one persistent launch (FLCE_GRAD_LAUNCH=combined)
+// or in two back-to-back launches (split, the default).
+bool grad_combined() {
+  const char* s = std::getenv("FLCE_GRAD_LAUNCH");
+  return s && std::strcmp(s, "combined") == 0;
+}
+
+TcProblem make_problem(const Engine& eg, int M, int N, int K, int a_mn, int b_mn, int epi, int m_fastest) {
   TcProblem P;
   std::memset(&P, 0, sizeof(P));
   P.M = M;
   P.N = N;
   P.K = K;
-  P.tiles_m = (int)ceil_div(M, TC_BM);
+  P.tiles_m = (int)ceil_div(M, eg.bm);
   P.tiles_n = (int)ceil_div(N, TC_BN);
   P.kblocks = (int)ceil_div(K, TC_BK);
   P.a_mn = a_mn;
@@ -277,12 +322,18 @@ TcProblem make_problem(int M, int N, int K, int a_mn, int b_mn, int epi, int m_f
   return P;
 }
 
-void launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
-               const CUtensorMap& b1, const TcParams& prm, int sms, cudaStream_t stream) {
+void launch_tc(const Engine& eg, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+               const CUtensorMap& b1, const TcParams& prm, const DeviceCtx* dev, cudaStream_t stream) {
+  const int sms = dev->sms;
   int64_t tiles = (int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n;
   if (prm.nprob > 1) tiles += (int64_t)prm.prob[1].tiles_m * prm.prob[1].tiles_n;
-  const int grid = (int)std::min<int64_t>(sms, tiles);
-  tc_gemm_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
+  if (eg.pair) {
+    const int pairs = (int)std::min<int64_t>(dev->pairs, tiles);
+    tc_gemm_pair_kernel<<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
+  } else {
+    const int grid = (int)std::min<int64_t>(sms, tiles);
+    tc_gemm_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
+  }
 }
 
 // ------------------------------------------------------------------ FLCE
@@ -369,6 +420,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   if (st != FLCE_OK) return st;
 
   const int64_t ldx = X->stride[0], ldw = W->stride[0];
+  const Engine eg = engine();
   for (int64_t c = 0; c < pl.n_chunks; ++c) {
     const int64_t r0 = c * pl.chunk;
     const int rows = (int)std::min<int64_t>(pl.chunk, BT - r0);
@@ -381,15 +433,15 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       {
         CUtensorMap ta, tb, z;
         std::memset(&z, 0, sizeof(z));
-        if (!make_tmap(&ta, Xc, H, rows, ldx * 2, 64, TC_BM) || !make_tmap(&tb, Wp, H, V, ldw * 2, 64, TC_BN))
+        if (!make_tmap(&ta, Xc, H, rows, ldx * 2, 64, 128) || !make_tmap(&tb, Wp, H, V, ldw * 2, 64, eg.b_box_rows))
           return FLCE_ERR_CUDA;
         TcParams prm;
         std::memset(&prm, 0, sizeof(prm));
         prm.nprob = 1;
-        prm.prob[0] = make_problem(rows, (int)V, (int)H, 0, 0, EPI_LOGITS, 1);
+        prm.prob[0] = make_problem(eg, rows, (int)V, (int)H, 0, 0, EPI_LOGITS, 1);
         prm.lg = LogitsArgs{tgt_c, ignore_index, V, E, pl.lde, pm, ps, pl.ldp, zt};
         prm.err = dev->err;
-        st = L.run(1, [&] { launch_tc(ta, tb, z, z, prm, dev->sms, stream); });
+        st = L.run(1, [&] { launch_tc(eg, ta, tb, z, z, prm, dev, stream); });
         if (st != FLCE_OK) return st;
       }
     } else {
@@ -445,7 +497,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         if (!make_tmap(&tm[2 * np], E, V, rows, pl.lde * 2, 64, TC_BM) ||
             !make_tmap(&tm[2 * np + 1], Wp, H, V, ldw * 2, 64, 64))
           return FLCE_ERR_CUDA;
-        TcProblem P = make_problem(rows, (int)H, (int)V, 0, 1, EPI_STORE_BF16, 1);
+        TcProblem P = make_problem(eg, rows, (int)H, (int)V, 0, 1, EPI_STORE_BF16, 1);
         P.out = static_cast<__nv_bfloat16*>(grad_X->data) + r0 * grad_X->stride[0];
         P.ldo = grad_X->stride[0];
         prm.prob[np++] = P;
@@ -454,7 +506,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         if (!make_tmap(&tm[2 * np], E, V, rows, pl.lde * 2, 64, 64) ||
             !make_tmap(&tm[2 * np + 1], Xc, H, rows, ldx * 2, 64, 64))
           return FLCE_ERR_CUDA;
-        TcProblem P = make_problem((int)V, (int)H, rows, 1, 1, EPI_GRADW, 0);
+        TcProblem P = make_problem(eg, (int)V, (int)H, rows, 1, 1, EPI_GRADW, 0);
         P.out = grad_W->data;
         P.ldo = grad_W->stride[0];
         const bool last = c == pl.n_chunks - 1;
@@ -464,8 +516,24 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         P.ld_facc = H;
         prm.prob[np++] = P;
       }
-      prm.nprob = np;
-      st = L.run(4, [&] { launch_tc(tm[0], tm[1], tm[2], tm[3], prm, dev->sms, stream); });
+      if (np == 2 && !grad_combined()) {
+        // grad_X and grad_W as two launches: they contend for L2 when interleaved
+        TcParams p1 = prm;
+        p1.nprob = 1;
+        p1.prob[1] = TcProblem{};
+        TcParams p2 = prm;
+        p2.nprob = 1;
+        p2.prob[0] = prm.prob[1];
+        p2.prob[1] = TcProblem{};
+        CUtensorMap z;
+        std::memset(&z, 0, sizeof(z));
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream); });
+        if (st != FLCE_OK) return st;
+        st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream); });
+      } else {
+        prm.nprob = np;
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream); });
+      }
       if (st != FLCE_OK) return st;
     } else {
       float* E = static_cast<float*>(estore);
@@ -684,17 +752,18 @@ flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, in
   if (st != FLCE_OK) return st;
   CUtensorMap ta, tb, z;
   std::memset(&z, 0, sizeof(z));
-  const bool ok = (a_mn_major ? make_tmap(&ta, A, M, K, lda * 2, 64, 64) : make_tmap(&ta, A, K, M, lda * 2, 64, TC_BM)) &&
-                  (b_mn_major ? make_tmap(&tb, B, N, K, ldb * 2, 64, 64) : make_tmap(&tb, B, K, N, ldb * 2, 64, TC_BN));
+  const Engine eg = engine();
+  const bool ok = (a_mn_major ? make_tmap(&ta, A, M, K, lda * 2, 64, 64) : make_tmap(&ta, A, K, M, lda * 2, 64, 128)) &&
+                  (b_mn_major ? make_tmap(&tb, B, N, K, ldb * 2, 64, 64) : make_tmap(&tb, B, K, N, ldb * 2, 64, eg.b_box_rows));
   if (!ok) return FLCE_ERR_CUDA;
   TcParams prm;
   std::memset(&prm, 0, sizeof(prm));
   prm.nprob = 1;
-  prm.prob[0] = make_problem((int)M, (int)N, (int)K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, EPI_STORE_F32, 1);
+  prm.prob[0] = make_problem(eg, (int)M, (int)N, (int)K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, EPI_STORE_F32, 1);
   prm.prob[0].out = C;
   prm.prob[0].ldo = ldc;
   prm.err = dev->err;
-  launch_tc(ta, tb, z, z, prm, dev->sms, reinterpret_cast<cudaStream_t>(stream));
+  launch_tc(eg, ta, tb, z, z, prm, dev, reinterpret_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   if (env_debug() && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FLCE_ERR_CUDA;

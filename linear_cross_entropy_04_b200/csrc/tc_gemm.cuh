@@ -156,10 +156,20 @@ __device__ __forceinline__ void sched_tile(const TcParams& p, const TileSched& s
 // Each thread holds accumulator row `row` (tile-local 0..127) of tile (tm, tn).
 // taddr addresses column 0 of that row's 32-lane group in the ready accumulator.
 
-__device__ __forceinline__ void epi_logits(const TcParams& p, const TcProblem& P, int tm, int tn,
-                                           int row, uint32_t taddr, uint64_t* tmem_empty_bar) {
+// Hands the accumulator back to the MMA issuer once this thread's reads are done.
+struct ReleaseLocal {  // 1-CTA engine: all 128 epilogue threads arrive
+  uint64_t* bar;
+  __device__ __forceinline__ void operator()() const {
+    tc_fence_before();
+    mbar_arrive(bar);
+  }
+};
+
+template <typename Release>
+__device__ __forceinline__ void epi_logits(const TcParams& p, const TcProblem& P, int64_t r_base, int tn,
+                                           int row, uint32_t taddr, const Release& release) {
   const LogitsArgs& g = p.lg;
-  const int64_t r = (int64_t)tm * TC_BM + row;
+  const int64_t r = r_base + row;
   const bool row_ok = r < P.M;
   const int64_t n0 = (int64_t)tn * TC_BN;
   const int ncols = (int)((g.V - n0) < TC_BN ? (g.V - n0) : TC_BN);
@@ -216,8 +226,7 @@ __device__ __forceinline__ void epi_logits(const TcParams& p, const TcProblem& P
     }
   }
   // the accumulator is no longer needed: hand it back to the MMA warp
-  tc_fence_before();
-  mbar_arrive(tmem_empty_bar);
+  release();
   if (row_ok) {
     g.part_m[(int64_t)tn * g.ldp + r] = mx;
     g.part_s[(int64_t)tn * g.ldp + r] = s;
@@ -225,9 +234,10 @@ __device__ __forceinline__ void epi_logits(const TcParams& p, const TcProblem& P
   }
 }
 
-__device__ __forceinline__ void epi_store(const TcProblem& P, int tm, int tn, int row,
-                                          uint32_t taddr, uint64_t* tmem_empty_bar) {
-  const int64_t r = (int64_t)tm * TC_BM + row;
+template <typename Release>
+__device__ __forceinline__ void epi_store(const TcProblem& P, int64_t r_base, int tn, int row,
+                                          uint32_t taddr, const Release& release) {
+  const int64_t r = r_base + row;
   const bool row_ok = r < P.M;
   const int64_t n0 = (int64_t)tn * TC_BN;
   const int ncols = (int)((P.N - n0) < TC_BN ? (P.N - n0) : TC_BN);
@@ -237,10 +247,7 @@ __device__ __forceinline__ void epi_store(const TcProblem& P, int tm, int tn, in
     __syncwarp();
     tmem_ld_32x32(taddr + c * 32, v);
     tmem_ld_wait();
-    if (c == TC_BN / 32 - 1) {
-      tc_fence_before();
-      mbar_arrive(tmem_empty_bar);
-    }
+    if (c == TC_BN / 32 - 1) release();
     if (!row_ok || c * 32 >= ncols) continue;
     const bool full = c * 32 + 32 <= ncols;
     const int64_t col0 = n0 + c * 32;
@@ -479,10 +486,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * TC_BN;
+      const ReleaseLocal rel{&tempty_bar[acc]};
       if (P.epi == EPI_LOGITS)
-        epi_logits(p, P, tm, tn, row, taddr, &tempty_bar[acc]);
+        epi_logits(p, P, (int64_t)tm * TC_BM, tn, row, taddr, rel);
       else
-        epi_store(P, tm, tn, row, taddr, &tempty_bar[acc]);
+        epi_store(P, (int64_t)tm * TC_BM, tn, row, taddr, rel);
     }
   }
 
