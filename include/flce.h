@@ -172,6 +172,34 @@ FLCE_API flce_status flce_cross_entropy(const flce_tensor* logits, const flce_te
                                const flce_options* opt);
 
 /*
+ * flce_cross_entropy without any device allocation. The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory where they compute the loss (while a CUDA graph is being
+ * captured around them, inside a host that owns all device memory through its
+ * own allocator, or in a loop where an allocation and the synchronisation it
+ * may bring are not allowed).
+ *   Arguments and results are those of flce_cross_entropy (opt is not taken:
+ *   the mean uses this call's own count of non-ignored rows). The caller still
+ *   provides logits, target, loss and grad_logits (which may be the logits).
+ *   Scratch comes from one fixed array of 8 MiB in device memory that every
+ *   GPU loading the library holds until the process exits. It needs about
+ *   8 * ceil(V / 1024) + 12 bytes per row (round BT up to a multiple of 32
+ *   for the first term), e.g. up to ~8200 rows at V = 128256; larger problems
+ *   return FLCE_ERR_WORKSPACE_TOO_SMALL before any GPU work.
+ *   The first call on a device looks up the array's device address (a CUDA
+ *   runtime query, no allocation); make that first call before any stream
+ *   capture. All calls share the array and it keeps the last call's contents;
+ *   every value a call reads from it is written earlier in the same call.
+ *   Calls that overlap on the GPU (on different streams, or from different
+ *   threads without ordering) race on the array: order them.
+ * Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+FLCE_API flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const flce_tensor* target,
+                                                int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                                                flce_tensor* grad_logits, flce_stream_t stream);
+
+/*
+ * Plain bf16 GEMM on the library's tcgen05 engine,/*
  * Plain bf16 GEMM on the library's tcgen05 engine, for testing that engine
  * on its own: C[M,N] (f32, row-major, ldc) = sum_k A(m,k) * B(n,k).
  * A is [M,K] row-major (a_mn_major = 0, lda >= K) or [K,M] row-major

@@ -74,6 +74,8 @@ _SIGS = {
                                         ctypes.c_void_p]),
     "flce_cross_entropy": (ctypes.c_int, [_P(FlceTensor), _P(FlceTensor), ctypes.c_int64, ctypes.c_int32,
                                           _P(FlceTensor), _P(FlceTensor), ctypes.c_void_p, _P(FlceOptions)]),
+    "flce_cross_entropy_noalloc": (ctypes.c_int, [_P(FlceTensor), _P(FlceTensor), ctypes.c_int64, ctypes.c_int32,
+                                                  _P(FlceTensor), _P(FlceTensor), ctypes.c_void_p]),
     "flce_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]),

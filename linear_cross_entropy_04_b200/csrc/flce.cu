@@ -668,6 +668,140 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   });
 }
 
+// ------------------------------------------------------------------ CE without allocation
+// Some callers cannot allocate device memory at the point where they need the
+// loss: code running while a CUDA graph is being captured around it, hosts
+// that hand all device memory to their own allocator and forbid outside
+// allocations, or real-time loops where an allocation (and the implicit
+// synchronisation it may bring) is not allowed. For them,
+// flce_cross_entropy_noalloc keeps its scratch in the fixed device array
+// below instead of asking for a workspace. The array is part of the library
+// image, so every GPU that loads the library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+  bool init = false;
+  bool supported = false;
+  uint8_t* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  uint32_t* err = nullptr;     // device address of the error word on this device
+};
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kMaxDevices];
+
+// Once per device, with that device current: look up the device addresses of
+// the scratch array and the error word. (In host code the array's name is only
+// a host-side stand-in; the kernels must be given the address found here.)
+flce_status noalloc_device(NoAllocDevice** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FLCE_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    d.supported = major == 10 && minor == 0;
+    if (d.supported) {
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.scratch), g_noalloc_scratch) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_err_word) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+    }
+    d.init = true;
+  }
+  if (!d.supported) return FLCE_ERR_UNSUPPORTED_DEVICE;
+  *out = &d;
+  return FLCE_OK;
+}
+
+flce_status run_ce_noalloc(const flce_tensor* Z, const flce_tensor* target, int64_t ignore_index,
+                           int32_t reduction, flce_tensor* loss, flce_tensor* grad, cudaStream_t stream) {
+  if (!Z || !target || !loss) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_MEAN && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  const int32_t dt = Z->dtype;
+  if (dt != FLCE_BF16 && dt != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
+  if (Z->ndim != 2) return FLCE_ERR_INVALID_ARG;
+  const int64_t BT = Z->shape[0], V = Z->shape[1];
+  if (BT < 0 || V <= 0 || BT >= (1ll << 31) || V >= (1ll << 31)) return FLCE_ERR_INVALID_ARG;
+  if (BT > 0 && !check_matrix(Z, dt, BT, V)) return FLCE_ERR_INVALID_ARG;
+  if (target->dtype != FLCE_I64 || target->ndim != 1 || target->shape[0] != BT ||
+      (BT > 0 && (!target->data || target->stride[0] != 1)))
+    return FLCE_ERR_INVALID_ARG;
+  if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
+      (loss->ndim == 1 && loss->shape[0] != 1))
+    return FLCE_ERR_INVALID_ARG;
+  const int esz = dtype_size(dt);
+  if (BT > 0 && (!is_aligned(Z->data, 16) || (Z->stride[0] * esz) % 16)) return FLCE_ERR_INVALID_ARG;
+  if (grad && BT > 0) {
+    if (!check_matrix(grad, dt, BT, V)) return FLCE_ERR_INVALID_ARG;
+    if (!is_aligned(grad->data, 16) || (grad->stride[0] * esz) % 16) return FLCE_ERR_INVALID_ARG;
+  }
+  // scratch plan; sizes beyond the fixed array are refused before any GPU work
+  const int shift = 10;
+  const int64_t ntile = ceil_div(V, 1 << shift), ldp = round_up(std::max<int64_t>(BT, 1), 32);
+  size_t o = 0;
+  const size_t off_nv = o; o = align256(o + 8);
+  const size_t off_rl = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_lse = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_zt = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_pm = o; o = align256(o + (size_t)ntile * ldp * 4);
+  const size_t off_ps = o; o = align256(o + (size_t)ntile * ldp * 4);
+  if (o > kNoAllocScratchBytes) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  NoAllocDevice* d = nullptr;
+  flce_status st = noalloc_device(&d);
+  if (st != FLCE_OK) return st;
+  if (BT == 0) return cudaMemsetAsync(loss->data, 0, 4, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  // Every value read from the scratch below is written earlier in the same
+  // call (count, partials, per-row values), so what a previous call left in
+  // the array never leaks into this one and nothing needs clearing first.
+  uint8_t* b = d->scratch;
+  int64_t* nv = reinterpret_cast<int64_t*>(b + off_nv);
+  float* rl = reinterpret_cast<float*>(b + off_rl);
+  float* lse = reinterpret_cast<float*>(b + off_lse);
+  float* zt = reinterpret_cast<float*>(b + off_zt);
+  float* pm = reinterpret_cast<float*>(b + off_pm);
+  float* ps = reinterpret_cast<float*>(b + off_ps);
+  const int64_t* tgt = static_cast<const int64_t*>(target->data);
+  count_valid_kernel<<<1, 1024, 0, stream>>>(tgt, BT, V, ignore_index, nv, d->err);
+  const int64_t warps = BT * ntile;
+  if (dt == FLCE_BF16) {
+    CePartialArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data), Z->stride[0], tgt, ignore_index, V,
+                                   pm, ps, ldp, zt, (int)BT, (int)ntile, shift};
+    ce_partials_kernel<__nv_bfloat16><<<(unsigned)ceil_div(warps, 8), 256, 0, stream>>>(a);
+  } else {
+    CePartialArgs<float> a{static_cast<const float*>(Z->data), Z->stride[0], tgt, ignore_index, V,
+                           pm, ps, ldp, zt, (int)BT, (int)ntile, shift};
+    ce_partials_kernel<float><<<(unsigned)ceil_div(warps, 8), 256, 0, stream>>>(a);
+  }
+  for (int64_t r0 = 0; r0 < BT; r0 += 65535 * 32) {
+    const int rows = (int)std::min<int64_t>(65535 * 32, BT - r0);
+    CombineArgs a{tgt + r0, ignore_index, V, rows, (int)ntile, ldp, pm + r0, ps + r0, zt + r0, rl + r0, lse + r0, nv, reduction};
+    combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a);
+  }
+  if (grad) {
+    for (int64_t r0 = 0; r0 < BT; r0 += 65535) {
+      const int rows = (int)std::min<int64_t>(65535, BT - r0);
+      const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
+      if (dt == FLCE_BF16) {
+        CeGradArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
+                                    static_cast<__nv_bfloat16*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
+                                    tgt + r0, ignore_index, V, lse + r0, nv, reduction};
+        ce_grad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
+      } else {
+        CeGradArgs<float> a{static_cast<const float*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
+                            static_cast<float*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
+                            tgt + r0, ignore_index, V, lse + r0, nv, reduction};
+        ce_grad_kernel<float><<<grid, 256, 0, stream>>>(a);
+      }
+    }
+  }
+  finalize_loss_kernel<<<1, 1024, 0, stream>>>(rl, BT, nv, reduction, static_cast<float*>(loss->data));
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace flce
 
@@ -734,6 +868,17 @@ flce_status flce_cross_entropy(const flce_tensor* logits, const flce_tensor* tar
   try {
     return run_ce(logits, target, ignore_index, reduction, loss, grad_logits,
                   reinterpret_cast<cudaStream_t>(stream), opt);
+  } catch (...) {
+    return FLCE_ERR_CUDA;
+  }
+}
+
+flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const flce_tensor* target,
+                                       int64_t ignore_index, int32_t reduction, flce_tensor* loss,
+                                       flce_tensor* grad_logits, flce_stream_t stream) {
+  try {
+    return run_ce_noalloc(logits, target, ignore_index, reduction, loss, grad_logits,
+                          reinterpret_cast<cudaStream_t>(stream));
   } catch (...) {
     return FLCE_ERR_CUDA;
   }
