@@ -318,6 +318,28 @@ __global__ void __launch_bounds__(1024) finalize_loss_kernel(const float* __rest
   }
 }
 
+// ------------------------------------------------------------------ split-K sum
+// out[r, h] = bf16(sum over s = 0..S-1 of part[s * stride + r * H + h]), in
+// that fixed order, so a split-K result does not depend on launch timing.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, int S,
+                                                            int64_t stride, int rows, int H,
+                                                            __nv_bfloat16* __restrict__ out, int64_t ldo) {
+  const int64_t n4 = (int64_t)rows * H / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i * 4;
+    const int64_t r = e / H, h = e % H;
+    float4 acc = reinterpret_cast<const float4*>(part + e)[0];
+    for (int s = 1; s < S; ++s) {
+      const float4 v = reinterpret_cast<const float4*>(part + s * stride + e)[0];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(acc.x, acc.y);
+    o.y = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(out + r * ldo + h) = o;
+  }
+}
+
 // ------------------------------------------------------------------ SIMT fp32
 // C(m, n) = sum_k A(m, k) * B(n, k) with A(m, k) = A[m*sam + k*sak] and
 // B(n, k) = B[n*sbn + k*sbk]. 64 x 64 tiles, 256 threads, 4 x 4 per thread.

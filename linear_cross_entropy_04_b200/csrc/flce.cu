@@ -130,13 +130,14 @@ flce_status device_ctx(DeviceCtx** out) {
 
 // bf16 2-D tensor map: dims {inner, outer}, row pitch in bytes, box {bi, bo}, 128B swizzle.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-               uint64_t pitch_bytes, uint32_t bi, uint32_t bo) {
+               uint64_t pitch_bytes, uint32_t bi, uint32_t bo,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {bi, bo};
   cuuint32_t estr[2] = {1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -153,14 +154,57 @@ bool check_matrix(const flce_tensor* t, int32_t dtype, int64_t rows, int64_t col
   return true;
 }
 
+// Split-K factor for a problem of `tiles` output tiles and `kblocks` K-blocks
+// on `units` concurrent workers (CTA pairs): the smallest S that minimises the
+// number of tile-waves per unit of work, ceil(tiles * S / units) / S, keeping
+// at least 32 K-blocks per split. S = 1 when splitting does not help.
+int choose_ksplit(int64_t tiles, int64_t kblocks, int64_t units) {
+  int best_s = 1;
+  double best = (double)ceil_div(tiles, units);
+  for (int S = 2; S <= 8 && kblocks / S >= 32; ++S) {
+    const double w = (double)ceil_div(tiles * S, units) / S;
+    if (w < best - 1e-9) {
+      best = w;
+      best_s = S;
+    }
+  }
+  // every split must own at least one K-block
+  const int64_t kps = ceil_div(kblocks, best_s);
+  return (int)ceil_div(kblocks, kps);
+}
+
+// grad_X split-K partial buffer (fp32 elements) the plan reserves: the largest
+// S * rows * H over the full and the last chunk, for the CTA-pair engine on a
+// B200 (74 pairs). A device with fewer pairs gets S clamped to fit.
+// Split-K for grad_X is opt-in (FLCE_GRADX_SPLITK=1): under the B200's power
+// cap the step is power-bound, so filling idle SMs did not shorten it, and
+// the partial buffer costs S * chunk_rows * H * 4 bytes of workspace.
+bool gradx_splitk_enabled() {
+  const char* s = std::getenv("FLCE_GRADX_SPLITK");
+  return s && s[0] == '1';
+}
+
+int64_t gradx_partial_elems(int64_t BT, int64_t H, int64_t V, int64_t chunk) {
+  if (BT <= 0 || !gradx_splitk_enabled()) return 0;
+  const int64_t last = BT - (ceil_div(BT, chunk) - 1) * chunk;
+  int64_t best = 0;
+  for (int64_t rows : {std::min(chunk, BT), last}) {
+    const int64_t tiles = ceil_div(rows, 256) * ceil_div(H, 256);
+    const int S = choose_ksplit(tiles, ceil_div(V, 64), 74);
+    if (S > 1) best = std::max(best, S * rows * H);
+  }
+  return best;
+}
+
 struct Plan {
   int64_t BT, H, V;
   int32_t dtype;
   int64_t chunk, n_chunks;
   int64_t tile_w;  // partial tile width (columns)
   int64_t ntile, lde, ldp;
-  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, total;
+  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, off_xpart, total;
   bool facc;
+  int64_t xpart_elems;  // grad_X split-K partials (fp32 elements)
 };
 
 flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want_gw,
@@ -207,6 +251,8 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
   p->off_ps = o; o = align256(o + (size_t)p->ntile * p->ldp * 4);
   p->off_e = o; o = align256(o + (size_t)chunk * p->lde * esz);
   p->off_facc = o; o = align256(o + (p->facc ? (size_t)V * H * 4 : 0));
+  p->xpart_elems = dtype == FLCE_BF16 ? gradx_partial_elems(BT, H, V, chunk) : 0;
+  p->off_xpart = o; o = align256(o + (size_t)p->xpart_elems * 4);
   p->total = o;
   return FLCE_OK;
 }
@@ -319,17 +365,31 @@ TcProblem make_problem(const Engine& eg, int M, int N, int K, int a_mn, int b_mn
   P.b_mn = b_mn;
   P.epi = epi;
   P.m_fastest = m_fastest;
+  P.ksplit = 1;
+  P.kb_per_split = P.kblocks;
   return P;
 }
 
+
+
+// Output map for the pair engine's TMA epilogue: bf16 [rows, cols] with row
+// pitch `ld` elements, written in unswizzled 32 x 32 boxes.
+bool make_out_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+  return make_tmap(m, base, cols, rows, ld * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 void launch_tc(const Engine& eg, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
-               const CUtensorMap& b1, const TcParams& prm, const DeviceCtx* dev, cudaStream_t stream) {
+               const CUtensorMap& b1, const TcParams& prm, const DeviceCtx* dev, cudaStream_t stream,
+               const CUtensorMap* c0 = nullptr, const CUtensorMap* c1 = nullptr) {
+  CUtensorMap zc;
+  std::memset(&zc, 0, sizeof(zc));
   const int sms = dev->sms;
   int64_t tiles = (int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n;
   if (prm.nprob > 1) tiles += (int64_t)prm.prob[1].tiles_m * prm.prob[1].tiles_n;
   if (eg.pair) {
     const int pairs = (int)std::min<int64_t>(dev->pairs, tiles);
-    tc_gemm_pair_kernel<<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
+    tc_gemm_pair_kernel<<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(a0, b0, a1, b1, c0 ? *c0 : zc,
+                                                                          c1 ? *c1 : zc, prm);
   } else {
     const int grid = (int)std::min<int64_t>(sms, tiles);
     tc_gemm_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
@@ -410,6 +470,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   float* ps = reinterpret_cast<float*>(base + pl.off_ps);
   void* estore = base + pl.off_e;
   float* facc = pl.facc ? reinterpret_cast<float*>(base + pl.off_facc) : nullptr;
+  float* xpart = pl.xpart_elems ? reinterpret_cast<float*>(base + pl.off_xpart) : nullptr;
   float* lse_out = opt ? opt->lse : nullptr;
   const int64_t* tgt = static_cast<const int64_t*>(target->data);
 
@@ -487,12 +548,14 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       const __nv_bfloat16* Xc = static_cast<const __nv_bfloat16*>(X->data) + r0 * ldx;
       const __nv_bfloat16* Wp = static_cast<const __nv_bfloat16*>(W->data);
       __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
-      CUtensorMap tm[4];
+      CUtensorMap tm[4], tc[2];
       std::memset(tm, 0, sizeof(tm));
+      std::memset(tc, 0, sizeof(tc));
       TcParams prm;
       std::memset(&prm, 0, sizeof(prm));
       prm.err = dev->err;
       int np = 0;
+      int gx_split = 1;
       if (want_gx) {
         if (!make_tmap(&tm[2 * np], E, V, rows, pl.lde * 2, 64, TC_BM) ||
             !make_tmap(&tm[2 * np + 1], Wp, H, V, ldw * 2, 64, 64))
@@ -500,6 +563,19 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         TcProblem P = make_problem(eg, rows, (int)H, (int)V, 0, 1, EPI_STORE_BF16, 1);
         P.out = static_cast<__nv_bfloat16*>(grad_X->data) + r0 * grad_X->stride[0];
         P.ldo = grad_X->stride[0];
+        if (!make_out_tmap(&tc[np], P.out, rows, H, grad_X->stride[0])) return FLCE_ERR_CUDA;
+        // few output tiles and a long K: split K so every SM (pair) has work
+        int S = choose_ksplit((int64_t)P.tiles_m * P.tiles_n, P.kblocks, eg.pair ? dev->pairs : dev->sms);
+        while (S > 1 && (int64_t)S * rows * H > pl.xpart_elems) --S;
+        if (S > 1) {
+          P.kb_per_split = (int)ceil_div(P.kblocks, S);
+          P.ksplit = (int)ceil_div(P.kblocks, P.kb_per_split);
+          P.epi = EPI_STORE_F32;
+          P.out = xpart;
+          P.ldo = H;
+          P.split_stride = (int64_t)rows * H;
+          gx_split = P.ksplit;
+        }
         prm.prob[np++] = P;
       }
       if (want_gw) {
@@ -509,6 +585,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         TcProblem P = make_problem(eg, (int)V, (int)H, rows, 1, 1, EPI_GRADW, 0);
         P.out = grad_W->data;
         P.ldo = grad_W->stride[0];
+        if (!make_out_tmap(&tc[np], P.out, V, H, grad_W->stride[0])) return FLCE_ERR_CUDA;
         const bool last = c == pl.n_chunks - 1;
         if (!pl.facc) P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
         else P.gw_mode = c == 0 ? GW_STORE_F32 : (last ? GW_FINAL_F32 : GW_ADD_F32);
@@ -527,14 +604,24 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         p2.prob[1] = TcProblem{};
         CUtensorMap z;
         std::memset(&z, 0, sizeof(z));
-        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream); });
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0]); });
         if (st != FLCE_OK) return st;
-        st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream); });
+        st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1]); });
       } else {
         prm.nprob = np;
-        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream); });
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], &tc[1]); });
       }
       if (st != FLCE_OK) return st;
+      if (gx_split > 1) {
+        __nv_bfloat16* gx = static_cast<__nv_bfloat16*>(grad_X->data) + r0 * grad_X->stride[0];
+        const int64_t n4 = (int64_t)rows * H / 4;
+        const int blocks = (int)std::min<int64_t>(ceil_div(n4, 256), 8 * dev->sms);
+        st = L.run(4, [&] {
+          splitk_reduce_kernel<<<blocks, 256, 0, stream>>>(xpart, gx_split, (int64_t)rows * H, rows, (int)H, gx,
+                                                           grad_X->stride[0]);
+        });
+        if (st != FLCE_OK) return st;
+      }
     } else {
       float* E = static_cast<float*>(estore);
       if (want_gx) {

@@ -66,6 +66,14 @@ struct TcProblem {
   int gw_mode;         // GradWMode (EPI_GRADW)
   float* facc;         // fp32 grad_W accumulator (GW_*_F32 modes)
   int64_t ld_facc;
+  int ksplit;          // split-K factor (>= 1): tile t covers K-blocks of split t / (tiles_m*tiles_n)
+  int kb_per_split;    // K-blocks per split
+  int64_t split_stride;  // elements between the output slices of consecutive splits
+};
+
+// One unit of work: output tile (tm, tn) of problem `prob` over K-blocks [kb0, kb1).
+struct Tile {
+  int prob, tm, tn, kb0, kb1, split;
 };
 
 struct LogitsArgs {
@@ -101,14 +109,14 @@ __device__ __forceinline__ int rr_count(int ntiles, int cta, int G) {
 __device__ TileSched make_sched(const TcParams& p, int cta, int G) {
   TileSched s;
   const TcProblem& P0 = p.prob[0];
-  const int n0 = P0.tiles_m * P0.tiles_n;
+  const int n0 = P0.tiles_m * P0.tiles_n * P0.ksplit;
   s.n0_mine = rr_count(n0, cta, G);
   s.p1_begin = s.p1_end = 0;
   if (p.nprob < 2) return s;
   const TcProblem& P1 = p.prob[1];
-  const int64_t n1 = (int64_t)P1.tiles_m * P1.tiles_n;
+  const int64_t n1 = (int64_t)P1.tiles_m * P1.tiles_n * P1.ksplit;
   // per-tile cost in K-blocks, plus two for the epilogue and hand-offs
-  const int64_t c0 = P0.kblocks + 2, c1 = P1.kblocks + 2;
+  const int64_t c0 = P0.kb_per_split + 2, c1 = P1.kb_per_split + 2;
   const int64_t target = ((int64_t)n0 * c0 + n1 * c1) / G;
   int64_t before = 0, total = 0, mine = 0;
   for (int j = 0; j < G; ++j) {
@@ -132,24 +140,30 @@ __device__ __forceinline__ int sched_count(const TileSched& s) {
   return s.n0_mine + (s.p1_end - s.p1_begin);
 }
 
-__device__ __forceinline__ void sched_tile(const TcParams& p, const TileSched& s, int cta, int G,
-                                           int i, int& prob, int& tm, int& tn) {
+__device__ __forceinline__ Tile sched_tile(const TcParams& p, const TileSched& s, int cta, int G, int i) {
+  Tile T;
   int t;
   if (i < s.n0_mine) {
-    prob = 0;
+    T.prob = 0;
     t = cta + i * G;
   } else {
-    prob = 1;
+    T.prob = 1;
     t = s.p1_begin + (i - s.n0_mine);
   }
-  const TcProblem& P = p.prob[prob];
+  const TcProblem& P = p.prob[T.prob];
+  const int per_split = P.tiles_m * P.tiles_n;
+  T.split = t / per_split;
+  t -= T.split * per_split;
   if (P.m_fastest) {
-    tm = t % P.tiles_m;
-    tn = t / P.tiles_m;
+    T.tm = t % P.tiles_m;
+    T.tn = t / P.tiles_m;
   } else {
-    tn = t % P.tiles_n;
-    tm = t / P.tiles_n;
+    T.tn = t % P.tiles_n;
+    T.tm = t / P.tiles_n;
   }
+  T.kb0 = T.split * P.kb_per_split;
+  T.kb1 = min(P.kblocks, T.kb0 + P.kb_per_split);
+  return T;
 }
 
 // ------------------------------------------------------------ epilogues
@@ -235,7 +249,7 @@ __device__ __forceinline__ void epi_logits(const TcParams& p, const TcProblem& P
 }
 
 template <typename Release>
-__device__ __forceinline__ void epi_store(const TcProblem& P, int64_t r_base, int tn, int row,
+__device__ __forceinline__ void epi_store(const TcProblem& P, int64_t r_base, int tn, int split, int row,
                                           uint32_t taddr, const Release& release) {
   const int64_t r = r_base + row;
   const bool row_ok = r < P.M;
@@ -252,7 +266,7 @@ __device__ __forceinline__ void epi_store(const TcProblem& P, int64_t r_base, in
     const bool full = c * 32 + 32 <= ncols;
     const int64_t col0 = n0 + c * 32;
     if (P.epi == EPI_STORE_F32) {
-      float* dst = reinterpret_cast<float*>(P.out) + r * P.ldo + col0;
+      float* dst = reinterpret_cast<float*>(P.out) + split * P.split_stride + r * P.ldo + col0;
       if (full) {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
@@ -390,8 +404,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t kit = 0;  // K-blocks issued so far: stage kit % STAGES, phase (kit / STAGES) & 1
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        int pi, tm, tn;
-        sched_tile(p, sched, cta, G, i, pi, tm, tn);
+        const Tile T = sched_tile(p, sched, cta, G, i);
+        const int pi = T.prob, tm = T.tm, tn = T.tn;
         const TcProblem& P = p.prob[pi];
         const CUtensorMap* tA = pi == 0 ? &tmA0 : &tmA1;
         const CUtensorMap* tB = pi == 0 ? &tmB0 : &tmB1;
@@ -402,7 +416,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (P.a_mn) a_boxes = min(2, (P.M - m0 + 63) / 64);
         if (P.b_mn) b_boxes = min(4, (P.N - n0 + 63) / 64);
         const uint32_t bytes = (P.a_mn ? a_boxes * 8192 : TC_A_BYTES) + (P.b_mn ? b_boxes * 8192 : TC_B_BYTES);
-        for (int kb = 0; kb < P.kblocks; ++kb, ++kit) {
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++kit) {
           const int stage = kit % TC_STAGES;
           const uint32_t phase = (kit / TC_STAGES) & 1;
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -436,16 +450,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t kit = 0;
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        int pi, tm, tn;
-        sched_tile(p, sched, cta, G, i, pi, tm, tn);
-        const TcProblem& P = p.prob[pi];
+        const Tile T = sched_tile(p, sched, cta, G, i);
+        const TcProblem& P = p.prob[T.prob];
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
         if (!mbar_wait(&tempty_bar[acc], aph ^ 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * TC_BN;
         const uint32_t idesc = idesc_bf16_f32(P.a_mn, P.b_mn, TC_BM, TC_BN);
-        for (int kb = 0; kb < P.kblocks; ++kb, ++kit) {
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++kit) {
           const int stage = kit % TC_STAGES;
           const uint32_t phase = (kit / TC_STAGES) & 1;
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.err)) { ok = false; break; }
@@ -458,7 +471,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
             const uint64_t bd = P.b_mn ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb != T.kb0) || (k != 0));
           }
           tc_commit(&empty_bar[stage]);
         }
@@ -477,9 +490,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     const int row = q * 32 + lane;
     for (int i = 0; i < ntiles; ++i) {
-      int pi, tm, tn;
-      sched_tile(p, sched, cta, G, i, pi, tm, tn);
-      const TcProblem& P = p.prob[pi];
+      const Tile T = sched_tile(p, sched, cta, G, i);
+      const TcProblem& P = p.prob[T.prob];
+      const int tm = T.tm, tn = T.tn;
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
       const bool ok = mbar_wait(&tfull_bar[acc], aph, abort_flag, p.err);
@@ -490,7 +503,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (P.epi == EPI_LOGITS)
         epi_logits(p, P, (int64_t)tm * TC_BM, tn, row, taddr, rel);
       else
-        epi_store(P, (int64_t)tm * TC_BM, tn, row, taddr, rel);
+        epi_store(P, (int64_t)tm * TC_BM, tn, T.split, row, taddr, rel);
     }
   }
 

@@ -46,7 +46,52 @@ constexpr int T2_PREFETCH = FLCE_PAIR_PREFETCH;
 constexpr int T2_A_BYTES = T2_HALF * T2_BK * 2;  // 16 KB
 constexpr int T2_B_BYTES = T2_HALF * T2_BK * 2;  // 16 KB
 constexpr int T2_STAGE_BYTES = T2_A_BYTES + T2_B_BYTES;
-constexpr int T2_SMEM_BYTES = T2_STAGES * T2_STAGE_BYTES + 1024 + 256;
+constexpr int T2_STAGE_OUT_BYTES = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
+constexpr int T2_OUT_BYTES = 4 * 2 * T2_STAGE_OUT_BYTES;  // 4 epilogue warps x 2 boxes
+constexpr int T2_SMEM_BYTES = T2_STAGES * T2_STAGE_BYTES + T2_OUT_BYTES + 1024 + 256;
+
+// bf16 output tile through shared memory and TMA: each epilogue warp writes its
+// 32 rows in 32-column boxes, alternating two staging boxes, and one lane
+// stores (store = true) or adds (store = false, the add done in L2) each box.
+// Rows and columns outside the tensor map's extent are clipped by the TMA.
+template <typename Release>
+__device__ __forceinline__ void epi_bf16_tma(const CUtensorMap* tmC, bool store, int64_t M, int64_t N,
+                                             int64_t rwarp, int tn, uint32_t taddr, uint8_t* boxes,
+                                             uint32_t& issued, const Release& release) {
+  const int lane = threadIdx.x & 31;
+  const int n0 = tn * 256;
+  uint32_t v[32];
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    __syncwarp();
+    tmem_ld_32x32(taddr + c * 32, v);
+    tmem_ld_wait();
+    if (c == 7) release();
+    if (rwarp >= M || n0 + c * 32 >= N) continue;  // whole box outside: warp-uniform
+    uint8_t* box = boxes + (issued & 1) * T2_STAGE_OUT_BYTES;
+    if (issued >= 2) {
+      if (lane == 0) bulk_wait_group_read<1>();  // the box written two stores ago is free again
+      __syncwarp();
+    }
+    uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                          pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                          pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                          pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (store)
+        tma_store_2d(tmC, box, n0 + c * 32, (int32_t)rwarp);
+      else
+        tma_reduce_add_2d(tmC, box, n0 + c * 32, (int32_t)rwarp);
+      bulk_commit_group();
+    }
+    ++issued;
+  }
+}
 
 struct ReleasePair {  // 2-CTA engine: one arrival per epilogue warp on the leader's barrier
   uint32_t leader_bar;  // shared::cluster address
@@ -60,11 +105,13 @@ struct ReleasePair {  // 2-CTA engine: one arrival per epilogue warp on the lead
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
                         const __grid_constant__ TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + T2_STAGES * T2_STAGE_BYTES);
+  uint8_t* out_boxes = smem + T2_STAGES * T2_STAGE_BYTES;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(out_boxes + T2_OUT_BYTES);
   uint64_t* empty_bar = full_bar + T2_STAGES;
   uint64_t* tfull_bar = empty_bar + T2_STAGES;
   uint64_t* tempty_bar = tfull_bar + 2;
@@ -118,14 +165,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       uint32_t kit = 0;
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        int pi, tm, tn;
-        sched_tile(p, sched, pair, G, i, pi, tm, tn);
+        const Tile T = sched_tile(p, sched, pair, G, i);
+        const int pi = T.prob, tm = T.tm, tn = T.tn;
         const TcProblem& P = p.prob[pi];
         const CUtensorMap* tA = pi == 0 ? &tmA0 : &tmA1;
         const CUtensorMap* tB = pi == 0 ? &tmB0 : &tmB1;
         const int am0 = tm * T2_BM + (int)rank * T2_HALF;  // this CTA's rows of A
         const int bn0 = tn * T2_BN + (int)rank * T2_HALF;  // this CTA's rows of B
-        for (int kb = 0; kb < P.kblocks; ++kb, ++kit) {
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++kit) {
           const int stage = kit % T2_STAGES;
           const uint32_t phase = (kit / T2_STAGES) & 1;
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -149,7 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             tma_load_2d_pair(sB + 8192, tB, fb, bn0 + 64, k0);
           }
           // warm L2 for a later K-block so the load above it finds its data there
-          if (T2_PREFETCH > 0 && kb + T2_PREFETCH < P.kblocks) {
+          if (T2_PREFETCH > 0 && kb + T2_PREFETCH < T.kb1) {
             const int kp = k0 + T2_PREFETCH * T2_BK;
             if (!P.a_mn) {
               tma_prefetch_2d(tA, kp, am0);
@@ -180,16 +227,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       uint32_t kit = 0;
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        int pi, tm, tn;
-        sched_tile(p, sched, pair, G, i, pi, tm, tn);
-        const TcProblem& P = p.prob[pi];
+        const Tile T = sched_tile(p, sched, pair, G, i);
+        const TcProblem& P = p.prob[T.prob];
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1;
         if (!mbar_wait(&tempty_bar[acc], aph ^ 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * T2_BN;
         const uint32_t idesc = idesc_bf16_f32(P.a_mn, P.b_mn, T2_BM, T2_BN);
-        for (int kb = 0; kb < P.kblocks; ++kb, ++kit) {
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++kit) {
           const int stage = kit % T2_STAGES;
           const uint32_t phase = (kit / T2_STAGES) & 1;
           if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.err)) { ok = false; break; }
@@ -202,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                                        : smem_desc_sw128(a_base + k * 32, 16, 1024);
             const uint64_t bd = P.b_mn ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
-            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb != T.kb0) || (k != 0));
           }
           tc_commit_pair_mc(&empty_bar[stage], 0x3);
         }
@@ -219,10 +265,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     // ---------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    uint8_t* my_boxes = out_boxes + (warp - 2) * 2 * T2_STAGE_OUT_BYTES;
+    uint32_t issued = 0;  // TMA output boxes this warp has issued
     for (int i = 0; i < ntiles; ++i) {
-      int pi, tm, tn;
-      sched_tile(p, sched, pair, G, i, pi, tm, tn);
-      const TcProblem& P = p.prob[pi];
+      const Tile T = sched_tile(p, sched, pair, G, i);
+      const TcProblem& P = p.prob[T.prob];
+      const int tm = T.tm, tn = T.tn;
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
       const bool ok = mbar_wait(&tfull_bar[acc], aph, abort_flag, p.err, FLCE_EPI_BACKOFF_NS);
@@ -231,11 +279,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * T2_BN;
       const ReleasePair rel{mapa_shared(smem_u32(&tempty_bar[acc]), 0)};
       const int64_t r_base = (int64_t)tm * T2_BM + rank * T2_HALF;
+      const bool tma_out = P.epi == EPI_STORE_BF16 ||
+                           (P.epi == EPI_GRADW && (P.gw_mode == GW_STORE_BF16 || P.gw_mode == GW_ADD_BF16));
       if (P.epi == EPI_LOGITS)
         epi_logits(p, P, r_base, tn, row, taddr, rel);
+      else if (tma_out)
+        epi_bf16_tma(T.prob == 0 ? &tmC0 : &tmC1, P.epi == EPI_STORE_BF16 || P.gw_mode == GW_STORE_BF16, P.M, P.N,
+                     r_base + q * 32, tn, taddr, my_boxes, issued, rel);
       else
-        epi_store(P, r_base, tn, row, taddr, rel);
+        epi_store(P, r_base, tn, T.split, row, taddr, rel);
     }
+    // every output box must be written before the CTA exits
+    if (lane == 0 && issued > 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();
