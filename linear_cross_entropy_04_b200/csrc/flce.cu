@@ -345,11 +345,18 @@ Engine engine() {
   return Engine{true, T2_BM, T2_HALF};
 }
 
-// grad_X and grad_W of a chunk in one persistent launch (FLCE_GRAD_LAUNCH=combined)
-// or in two back-to-back launches (split, the default).
-bool grad_combined() {
+// grad_X and grad_W of a chunk in one persistent launch ("combined") or in two
+// back-to-back launches ("split"). Split avoids the two problems contending for
+// L2; combined lets grad_W tiles fill the SMs that grad_X's few output tiles
+// leave idle. The default picks combined when grad_X alone would keep less
+// than 80% of the workers busy over its waves (measured crossover on B200);
+// FLCE_GRAD_LAUNCH=split|combined forces one.
+bool grad_combined(int64_t gradx_tiles, int64_t units) {
   const char* s = std::getenv("FLCE_GRAD_LAUNCH");
-  return s && std::strcmp(s, "combined") == 0;
+  if (s && std::strcmp(s, "combined") == 0) return true;
+  if (s && std::strcmp(s, "split") == 0) return false;
+  const double eff = (double)gradx_tiles / (double)(ceil_div(gradx_tiles, units) * units);
+  return eff < 0.8;
 }
 
 TcProblem make_problem(const Engine& eg, int M, int N, int K, int a_mn, int b_mn, int epi, int m_fastest) {
@@ -593,7 +600,8 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         P.ld_facc = H;
         prm.prob[np++] = P;
       }
-      if (np == 2 && !grad_combined()) {
+      const int64_t units = eg.pair ? dev->pairs : dev->sms;
+      if (np == 2 && !grad_combined((int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n * prm.prob[0].ksplit, units)) {
         // grad_X and grad_W as two launches: they contend for L2 when interleaved
         TcParams p1 = prm;
         p1.nprob = 1;
