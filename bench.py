@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--grad-w-accum", default="output", choices=["output", "fp32"])
+    ap.add_argument("--path", default="flce", choices=["flce", "ce"],
+                    help="flce: the fused lm_head + loss step (default); ce: cross-entropy of given logits")
     return ap.parse_args()
 
 
@@ -224,12 +226,82 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- logits-given CE
+
+def run_ce(args):
+    """Cross-entropy of given logits [BT, V] (the paper review's CrossEntropy
+    kernel: online softmax, gradient written over the logits) against the
+    plain PyTorch cross_entropy + backward on the same bf16 logits."""
+    import torch
+    import torch.nn.functional as F
+
+    import linear_cross_entropy_04_b200 as flce
+    from linear_cross_entropy_04_b200.inputs import WORKLOADS, draw_targets
+
+    import numpy as np
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    z0 = (torch.randn(w.BT, w.V, device=dev, generator=g) * 1.28).to(torch.bfloat16)
+    t = torch.from_numpy(draw_targets(np.random.default_rng(0), w.BT, w.V, w.targets, w.ignore_frac)).to(dev)
+    z = z0.clone()
+
+    def ours():
+        flce.cross_entropy(z, t, inplace=True)
+
+    def torch_ce():
+        zz = z0.detach().requires_grad_(True)
+        F.cross_entropy(zz, t, ignore_index=-100).backward()
+        return zz.grad
+
+    res = {}
+    for name, fn in (("ours", ours), ("torch", torch_ce)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        res[name] = {"ms_per_step": ms, "tokens_per_s": w.BT / (ms / 1e3),
+                     "peak_extra_bytes": torch.cuda.max_memory_allocated(dev) - base}
+    # the library's CE workspace (taken from its own pool, invisible to torch's counters):
+    # N, per-row loss / lse / target logit, and per-(1024-column tile, row) max and sum-exp
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    ntile, ldp = -(-w.V // 1024), -(-w.BT // 32) * 32
+    lib_ws = a256(8) + 3 * a256(4 * w.BT) + 2 * a256(4 * ntile * ldp)
+    res["ours"]["peak_extra_bytes"] += lib_ws
+    res["ours"]["library_workspace_bytes"] = lib_ws
+    bytes_moved = 3 * w.BT * w.V * 2  # read z twice, write dz once (bf16)
+    line = {"metric": "CE (logits given) fwd+bwd tokens/s and peak extra memory", "value": res["ours"]["tokens_per_s"],
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": res["ours"]["ms_per_step"], "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": f"{w.name} logits", "BT": w.BT, "V": w.V},
+            "speedup_vs_torch": res["torch"]["ms_per_step"] / res["ours"]["ms_per_step"],
+            "memory_ratio_torch_over_ours": res["torch"]["peak_extra_bytes"] / max(res["ours"]["peak_extra_bytes"], 1),
+            "ours": res["ours"], "torch": res["torch"],
+            "roofline": {"bound": "hbm", "achieved": bytes_moved / (res["ours"]["ms_per_step"] / 1e3) / 1e9,
+                         "peak": load_peaks()["hbm_gbs"], "unit": "GB/s",
+                         "frac": bytes_moved / (res["ours"]["ms_per_step"] / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
+                         "traffic": None, "algorithmic_bytes": bytes_moved}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.path == "ce":
+        return run_ce(args)
 
     import torch
     import torch.distributed as dist

@@ -63,7 +63,8 @@ typedef enum {
 } flce_status;
 
 typedef enum { FLCE_F32 = 0, FLCE_BF16 = 1, FLCE_I64 = 2 } flce_dtype;
-typedef enum { FLCE_MEAN = 0, FLCE_SUM = 1 } flce_reduction;
+/* FLCE_NONE: `loss` is fp32 [BT] and receives the per-row losses (0 for ignored rows). */
+typedef enum { FLCE_MEAN = 0, FLCE_SUM = 1, FLCE_NONE = 2 } flce_reduction;
 
 /* Bits of the device error word. */
 #define FLCE_DEVERR_TARGET_RANGE 0x1u /* a target outside [0,V) that is not ignore_index */
@@ -101,6 +102,9 @@ typedef struct {
                                     flce_count_valid + an all-reduce). NULL = count locally. */
   float* row_loss;               /* optional DEVICE [BT] fp32: per-row losses l_i (0 if ignored) */
   float* lse;                    /* optional DEVICE [BT] fp32: per-row logsumexp of z_i */
+  const float* row_grad;         /* optional DEVICE [BT] fp32: upstream gradient per row; the
+                                    gradients are those of sum_i row_grad_i * l_i * (1/N or 1).
+                                    NULL = all ones. */
 } flce_options;
 
 typedef struct {
@@ -120,8 +124,9 @@ FLCE_API void flce_options_init(flce_options* opt);
  *   X       [BT,H]  bf16 or f32 (row-major)
  *   W       [V,H]   same dtype as X
  *   target  [BT]    int64; rows equal to ignore_index are ignored
- *   reduction       FLCE_MEAN or FLCE_SUM
- *   loss    scalar  f32 (ndim 0, or ndim 1 with one element): written
+ *   reduction       FLCE_MEAN, FLCE_SUM or FLCE_NONE
+ *   loss    scalar  f32 (ndim 0, or ndim 1 with one element): written;
+ *                   for FLCE_NONE, f32 [BT]: the per-row losses
  *   grad_X  [BT,H]  same dtype as X, or NULL to skip: fully overwritten
  *   grad_W  [V,H]   same dtype as W, or NULL to skip: fully overwritten
  * bf16 runs the tcgen05 tensor-core path (fp32 accumulation, bf16 results,
@@ -164,7 +169,8 @@ FLCE_API flce_status flce_count_valid(const flce_tensor* target, int64_t V, int6
  *   logits [BT,V] bf16 or f32; target [BT] int64; loss scalar f32.
  *   grad_logits: same shape/dtype as logits, or NULL to skip. It may be the
  *   logits tensor itself (in-place gradient replacement).
- * opt may be NULL; only opt->n_valid, opt->row_loss and opt->lse are read.
+ * opt may be NULL; only opt->n_valid, opt->row_loss, opt->lse and opt->row_grad are read.
+ * FLCE_NONE as for flce_fwd_bwd (loss is f32 [BT]).
  */
 FLCE_API flce_status flce_cross_entropy(const flce_tensor* logits, const flce_tensor* target,
                                int64_t ignore_index, int32_t reduction, flce_tensor* loss,

@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("FLCE_LIBRARY") or os.path.join(PKG, "libflce.so")
 
 F32, BF16, I64 = 0, 1, 2
-MEAN, SUM = 0, 1
+MEAN, SUM, NONE = 0, 1, 2
 FLAG_SYNC_CHECK, FLAG_TIME_PHASES = 0x1, 0x2
 GRADW_ACCUM_OUTPUT, GRADW_ACCUM_FP32 = 0, 1
 DEVERR_TARGET_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
@@ -38,7 +38,8 @@ class FlceOptions(ctypes.Structure):
     _fields_ = [("chunk_rows", ctypes.c_int64), ("workspace_limit_bytes", ctypes.c_int64),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_int64),
                 ("grad_w_accum", ctypes.c_int32), ("flags", ctypes.c_int32),
-                ("n_valid", ctypes.c_void_p), ("row_loss", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+                ("n_valid", ctypes.c_void_p), ("row_loss", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("row_grad", ctypes.c_void_p)]
 
 
 class FlceStats(ctypes.Structure):

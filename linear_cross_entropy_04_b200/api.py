@@ -14,12 +14,12 @@ import torch
 
 from . import _binding as B
 
-_RED = {"mean": B.MEAN, "sum": B.SUM}
+_RED = {"mean": B.MEAN, "sum": B.SUM, "none": B.NONE}
 _ACC = {"output": B.GRADW_ACCUM_OUTPUT, "fp32": B.GRADW_ACCUM_FP32}
 
 
 def _options(chunk_rows=0, workspace_limit_bytes=0, grad_w_accum="output", flags=0,
-             n_valid=None, row_loss=None, lse=None, workspace=None):
+             n_valid=None, row_loss=None, lse=None, workspace=None, row_grad=None):
     o = B.FlceOptions()
     B.lib().flce_options_init(ctypes.byref(o))
     o.chunk_rows = int(chunk_rows)
@@ -29,6 +29,7 @@ def _options(chunk_rows=0, workspace_limit_bytes=0, grad_w_accum="output", flags
     o.n_valid = None if n_valid is None else n_valid.data_ptr()
     o.row_loss = None if row_loss is None else row_loss.data_ptr()
     o.lse = None if lse is None else lse.data_ptr()
+    o.row_grad = None if row_grad is None else row_grad.data_ptr()
     if workspace is not None:
         o.workspace = workspace.data_ptr()
         o.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -41,11 +42,15 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                chunk_rows: int = 0, workspace_limit_bytes: int = 0,
                                grad_w_accum: str = "output", n_valid: Optional[torch.Tensor] = None,
                                row_loss: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                               row_grad: Optional[torch.Tensor] = None,
                                flags: int = 0, stream=None, out=None, host_out=None,
                                return_stats: bool = False):
     """Loss, grad_X and grad_W of cross-entropy over X W^T in one call.
 
     X [BT, H] and W [V, H] (bf16 or fp32, CUDA), target [BT] int64.
+    reduction 'mean' | 'sum' | 'none' ('none': loss is the [BT] per-row losses).
+    row_grad [BT] fp32 scales each row's contribution to the gradients (the
+    upstream gradient of the per-row losses); default all ones.
     Tensors on the host are staged to the current CUDA device and the
     results copied back (the end-to-end path); nothing runs on the CPU.
     host_out = (loss, grad_X, grad_W) pinned host tensors receive them then.
@@ -62,10 +67,13 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     if out is not None:
         loss, gX, gW = out
     else:
-        loss = torch.empty((), dtype=torch.float32, device=X.device)
+        loss = torch.empty((X.shape[0],) if reduction == "none" else (), dtype=torch.float32, device=X.device)
         gX = torch.empty_like(X) if want_grad_X else None
         gW = torch.empty_like(W) if want_grad_W else None
-    o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags, n_valid, row_loss, lse)
+    if row_grad is not None:
+        row_grad = row_grad.to(device=X.device, dtype=torch.float32).contiguous()
+    o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags, n_valid, row_loss, lse,
+                 row_grad=row_grad)
     st = B.FlceStats()
     B.check(B.lib().flce_plan(X.shape[0], X.shape[1], W.shape[0], B.dtype_code(X), int(gW is not None),
                               ctypes.byref(o), ctypes.byref(st)), "flce_plan")
@@ -104,14 +112,17 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
 def cross_entropy(logits: torch.Tensor, target: torch.Tensor, ignore_index: int = -100,
                   reduction: str = "mean", want_grad: bool = True, inplace: bool = False,
                   n_valid: Optional[torch.Tensor] = None, row_loss: Optional[torch.Tensor] = None,
-                  lse: Optional[torch.Tensor] = None, stream=None):
+                  lse: Optional[torch.Tensor] = None, row_grad: Optional[torch.Tensor] = None, stream=None):
     """Cross-entropy of given logits [BT, V]; the gradient may replace the logits in place."""
-    loss = torch.empty((), dtype=torch.float32, device=logits.device)
+    loss = torch.empty((logits.shape[0],) if reduction == "none" else (), dtype=torch.float32,
+                       device=logits.device)
     grad = None
     if want_grad:
         grad = logits if inplace else torch.empty_strided(logits.size(), logits.stride(), dtype=logits.dtype,
                                                           device=logits.device)
-    o = _options(n_valid=n_valid, row_loss=row_loss, lse=lse)
+    if row_grad is not None:
+        row_grad = row_grad.to(device=logits.device, dtype=torch.float32).contiguous()
+    o = _options(n_valid=n_valid, row_loss=row_loss, lse=lse, row_grad=row_grad)
     tz, tt, tl = B.tensor(logits), B.tensor(target), B.tensor(loss)
     tg = B.tensor(grad) if grad is not None else None
     rc = B.lib().flce_cross_entropy(ctypes.byref(tz), ctypes.byref(tt), int(ignore_index), _RED[reduction],
@@ -167,8 +178,11 @@ def phase_times(reset: bool = True) -> dict:
 
 
 class _FLCEFunction(torch.autograd.Function):
-    """Forward computes the loss and both gradients at once (the gradients are
-    produced in the forward pass and handed back, scaled, in backward)."""
+    """'mean' / 'sum': the forward computes the loss and both gradients at
+    once, and backward hands them back scaled by the upstream gradient.
+    'none': the forward computes only the per-row losses; backward runs the
+    fused path again with the per-row upstream gradient (row_grad), so the
+    logits GEMM is done twice in exchange for never storing dlogits."""
 
     @staticmethod
     def forward(ctx, weight, inp, target, ignore_index, reduction, grad_w_accum):
@@ -176,17 +190,34 @@ class _FLCEFunction(torch.autograd.Function):
         X = inp.reshape(-1, shape[-1])
         if X.stride(-1) != 1 or (X.stride(0) % 8 and X.dtype == torch.bfloat16):
             X = X.contiguous()
+        t = target.reshape(-1)
+        ctx.shape = shape
+        ctx.reduction = reduction
+        ctx.ignore_index = ignore_index
+        ctx.grad_w_accum = grad_w_accum
+        if reduction == "none":
+            loss, _, _ = fused_linear_cross_entropy(X, weight, t, ignore_index=ignore_index, reduction="none",
+                                                    want_grad_X=False, want_grad_W=False)
+            ctx.save_for_backward(X, weight, t)
+            ctx.need = (ctx.needs_input_grad[1], ctx.needs_input_grad[0])
+            return loss.reshape(shape[:-1])
         loss, gX, gW = fused_linear_cross_entropy(
-            X, weight, target.reshape(-1), ignore_index=ignore_index, reduction=reduction,
+            X, weight, t, ignore_index=ignore_index, reduction=reduction,
             want_grad_X=ctx.needs_input_grad[1], want_grad_W=ctx.needs_input_grad[0],
             grad_w_accum=grad_w_accum)
         ctx.save_for_backward(gX if gX is not None else torch.empty(0), gW if gW is not None else torch.empty(0))
         ctx.has = (gX is not None, gW is not None)
-        ctx.shape = shape
         return loss
 
     @staticmethod
     def backward(ctx, grad_out):
+        if ctx.reduction == "none":
+            X, W, t = ctx.saved_tensors
+            want_x, want_w = ctx.need
+            _, gX, gW = fused_linear_cross_entropy(X, W, t, ignore_index=ctx.ignore_index, reduction="none",
+                                                   row_grad=grad_out.reshape(-1), want_grad_X=want_x,
+                                                   want_grad_W=want_w, grad_w_accum=ctx.grad_w_accum)
+            return gW, (gX.reshape(ctx.shape) if gX is not None else None), None, None, None, None
         gX, gW = ctx.saved_tensors
         hx, hw = ctx.has
         one = grad_out.numel() == 1 and bool(grad_out == 1)
@@ -199,12 +230,13 @@ class FusedLinearCrossEntropyLoss(torch.nn.Module):
     """loss_fn(lm_head.weight, input, target) -> scalar loss with autograd.
 
     input may be [BT, H] or [B, T, H]; target has the matching leading shape.
+    reduction 'none' returns the per-row losses with the leading shape.
     """
 
     def __init__(self, ignore_index: int = -100, reduction: str = "mean", grad_w_accum: str = "output"):
         super().__init__()
         if reduction not in _RED:
-            raise ValueError("reduction must be 'mean' or 'sum'")
+            raise ValueError("reduction must be 'mean', 'sum' or 'none'")
         self.ignore_index = ignore_index
         self.reduction = reduction
         self.grad_w_accum = grad_w_accum

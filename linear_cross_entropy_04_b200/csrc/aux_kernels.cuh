@@ -26,6 +26,7 @@ __device__ __forceinline__ bool target_valid(int64_t t, int64_t V, int64_t ignor
   return t != ignore_index && t >= 0 && t < V;
 }
 
+// 1/N for the mean reduction, 1 for sum and none.
 __device__ __forceinline__ float mean_scale(const int64_t* n_valid, int reduction) {
   if (reduction != 0) return 1.f;
   const int64_t n = *n_valid;
@@ -71,6 +72,7 @@ struct CombineArgs {
   float* lse_out;         // optional [rows] at chunk row 0
   const int64_t* n_valid;
   int reduction;
+  const float* row_grad;  // optional [rows] at chunk row 0: upstream gradient per row
 };
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   __syncthreads();
   if (row_ok) {
     const bool valid = target_valid(a.target[r], a.V, a.ignore_index);
-    const float scale = mean_scale(a.n_valid, a.reduction);
+    const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
     const float lse = sm_lse[lane];
     for (int j = w; j < a.ntile; j += 8) {
       float* pm = a.part_m + (int64_t)j * a.ldp + r;
@@ -171,6 +173,7 @@ struct DlogitsArgs {
   int tile_shift;         // log2 of the partial tile width
   const int64_t* n_valid;
   int reduction;
+  const float* row_grad;  // optional [rows] at chunk row 0
 };
 
 template <typename T>
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs<T> a) {
   if (c0 >= a.V) return;
   const int64_t t = a.target[r];
   const bool valid = target_valid(t, a.V, a.ignore_index);
-  const float scale = mean_scale(a.n_valid, a.reduction);
+  const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
   const float f = a.factor[(c0 >> a.tile_shift) * a.ldp + r];
   const T* s = a.src + r * a.lds + c0;
   T* d = a.e + r * a.lde + c0;
@@ -258,6 +261,7 @@ struct CeGradArgs {
   const float* lse;
   const int64_t* n_valid;
   int reduction;
+  const float* row_grad;  // optional [rows] at row 0
 };
 
 template <typename T>
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(256) ce_grad_kernel(CeGradArgs<T> a) {
   if (c0 >= a.V) return;
   const int64_t t = a.target[r];
   const bool valid = target_valid(t, a.V, a.ignore_index);
-  const float scale = mean_scale(a.n_valid, a.reduction);
+  const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
   const float ls = a.lse[r] * LOG2E_F;
   const T* s = a.z + r * a.ldz + c0;
   T* d = a.dz + r * a.ldd + c0;

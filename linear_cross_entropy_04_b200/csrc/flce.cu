@@ -410,7 +410,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
                      const flce_options* opt, flce_stats* stats) {
   // ---- host-side argument checks (nothing is enqueued before they pass)
   if (!X || !W || !target || !loss) return FLCE_ERR_INVALID_ARG;
-  if (reduction != FLCE_MEAN && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_MEAN && reduction != FLCE_SUM && reduction != FLCE_NONE) return FLCE_ERR_INVALID_ARG;
   const int32_t dt = X->dtype;
   if (dt != FLCE_BF16 && dt != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
   if (W->dtype != dt) return FLCE_ERR_UNSUPPORTED_DTYPE;
@@ -422,9 +422,15 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   if (target->dtype != FLCE_I64 || target->ndim != 1 || target->shape[0] != BT ||
       (BT > 0 && (!target->data || target->stride[0] != 1)))
     return FLCE_ERR_INVALID_ARG;
-  if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
-      (loss->ndim == 1 && loss->shape[0] != 1))
+  if (reduction == FLCE_NONE) {
+    // per-row losses: f32 [BT], contiguous
+    if (loss->dtype != FLCE_F32 || loss->ndim != 1 || loss->shape[0] != BT ||
+        (BT > 0 && (!loss->data || loss->stride[0] != 1)))
+      return FLCE_ERR_INVALID_ARG;
+  } else if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
+             (loss->ndim == 1 && loss->shape[0] != 1)) {
     return FLCE_ERR_INVALID_ARG;
+  }
   if (grad_X && (BT > 0 && !check_matrix(grad_X, dt, BT, H))) return FLCE_ERR_INVALID_ARG;
   if (grad_W && !check_matrix(grad_W, dt, V, H)) return FLCE_ERR_INVALID_ARG;
   if (dt == FLCE_BF16) {
@@ -436,7 +442,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   }
   const bool want_gx = grad_X != nullptr && BT > 0;
   const bool want_gw = grad_W != nullptr;
-  const bool need_rowloss = !(opt && opt->row_loss);
+  const bool need_rowloss = reduction != FLCE_NONE && !(opt && opt->row_loss);
   Plan pl;
   flce_status st = make_plan(BT, H, V, dt, want_gw, opt, need_rowloss, &pl);
   if (st != FLCE_OK) return st;
@@ -457,7 +463,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
 
   if (BT == 0) {
-    if (cudaMemsetAsync(loss->data, 0, 4, stream) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (reduction != FLCE_NONE && cudaMemsetAsync(loss->data, 0, 4, stream) != cudaSuccess) return FLCE_ERR_CUDA;
     if (want_gw && cudaMemset2DAsync(grad_W->data, grad_W->stride[0] * dtype_size(dt), 0,
                                      H * dtype_size(dt), V, stream) != cudaSuccess)
       return FLCE_ERR_CUDA;
@@ -471,7 +477,9 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   uint8_t* base = static_cast<uint8_t*>(ws.ptr);
   int64_t* nvalid_local = reinterpret_cast<int64_t*>(base + pl.off_nvalid);
   const int64_t* nvalid = (opt && opt->n_valid) ? opt->n_valid : nvalid_local;
-  float* row_loss = need_rowloss ? reinterpret_cast<float*>(base + pl.off_rowloss) : opt->row_loss;
+  float* row_loss = reduction == FLCE_NONE ? static_cast<float*>(loss->data)
+                    : need_rowloss ? reinterpret_cast<float*>(base + pl.off_rowloss) : opt->row_loss;
+  const float* row_grad = opt ? opt->row_grad : nullptr;
   float* zt = reinterpret_cast<float*>(base + pl.off_zt);
   float* pm = reinterpret_cast<float*>(base + pl.off_pm);
   float* ps = reinterpret_cast<float*>(base + pl.off_ps);
@@ -530,7 +538,8 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     // A3
     {
       CombineArgs a{tgt_c, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, ps, zt,
-                    row_loss + r0, lse_out ? lse_out + r0 : nullptr, nvalid, reduction};
+                    row_loss + r0, lse_out ? lse_out + r0 : nullptr, nvalid, reduction,
+                    row_grad ? row_grad + r0 : nullptr};
       st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
       if (st != FLCE_OK) return st;
     }
@@ -541,11 +550,13 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
       if (dt == FLCE_BF16) {
         __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
-        DlogitsArgs<__nv_bfloat16> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction};
+        DlogitsArgs<__nv_bfloat16> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction,
+                                     row_grad ? row_grad + r0 : nullptr};
         st = L.run(3, [&] { dlogits_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a); });
       } else {
         float* E = static_cast<float*>(estore);
-        DlogitsArgs<float> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction};
+        DlogitsArgs<float> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction,
+                             row_grad ? row_grad + r0 : nullptr};
         st = L.run(3, [&] { dlogits_kernel<float><<<grid, 256, 0, stream>>>(a); });
       }
       if (st != FLCE_OK) return st;
@@ -662,11 +673,13 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       }
     }
   }
-  st = L.run(5, [&] {
-    finalize_loss_kernel<<<1, 1024, 0, stream>>>(row_loss, BT, nvalid, reduction,
-                                                 static_cast<float*>(loss->data));
-  });
-  if (st != FLCE_OK) return st;
+  if (reduction != FLCE_NONE) {
+    st = L.run(5, [&] {
+      finalize_loss_kernel<<<1, 1024, 0, stream>>>(row_loss, BT, nvalid, reduction,
+                                                   static_cast<float*>(loss->data));
+    });
+    if (st != FLCE_OK) return st;
+  }
   if (stats) stats->kernel_launches = L.launches;
   return FLCE_OK;
 }
@@ -676,7 +689,7 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
                    int32_t reduction, flce_tensor* loss, flce_tensor* grad, cudaStream_t stream,
                    const flce_options* opt) {
   if (!Z || !target || !loss) return FLCE_ERR_INVALID_ARG;
-  if (reduction != FLCE_MEAN && reduction != FLCE_SUM) return FLCE_ERR_INVALID_ARG;
+  if (reduction != FLCE_MEAN && reduction != FLCE_SUM && reduction != FLCE_NONE) return FLCE_ERR_INVALID_ARG;
   const int32_t dt = Z->dtype;
   if (dt != FLCE_BF16 && dt != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
   if (Z->ndim != 2) return FLCE_ERR_INVALID_ARG;
@@ -686,9 +699,14 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   if (target->dtype != FLCE_I64 || target->ndim != 1 || target->shape[0] != BT ||
       (BT > 0 && (!target->data || target->stride[0] != 1)))
     return FLCE_ERR_INVALID_ARG;
-  if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
-      (loss->ndim == 1 && loss->shape[0] != 1))
+  if (reduction == FLCE_NONE) {
+    if (loss->dtype != FLCE_F32 || loss->ndim != 1 || loss->shape[0] != BT ||
+        (BT > 0 && (!loss->data || loss->stride[0] != 1)))
+      return FLCE_ERR_INVALID_ARG;
+  } else if (!loss->data || loss->dtype != FLCE_F32 || loss->ndim > 1 ||
+             (loss->ndim == 1 && loss->shape[0] != 1)) {
     return FLCE_ERR_INVALID_ARG;
+  }
   const int esz = dtype_size(dt);
   if (BT > 0 && (!is_aligned(Z->data, 16) || (Z->stride[0] * esz) % 16)) return FLCE_ERR_INVALID_ARG;
   if (grad && BT > 0) {
@@ -698,7 +716,10 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   DeviceCtx* dev = nullptr;
   flce_status st = device_ctx(&dev);
   if (st != FLCE_OK) return st;
-  if (BT == 0) return cudaMemsetAsync(loss->data, 0, 4, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  if (BT == 0) {
+    if (reduction == FLCE_NONE) return FLCE_OK;
+    return cudaMemsetAsync(loss->data, 0, 4, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  }
   const int shift = 10;
   const int64_t ntile = ceil_div(V, 1 << shift), ldp = round_up(BT, 32);
   size_t o = 0;
@@ -714,7 +735,9 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   uint8_t* b = static_cast<uint8_t*>(ws.ptr);
   int64_t* nv_local = reinterpret_cast<int64_t*>(b + off_nv);
   const int64_t* nv = (opt && opt->n_valid) ? opt->n_valid : nv_local;
-  float* rl = (opt && opt->row_loss) ? opt->row_loss : reinterpret_cast<float*>(b + off_rl);
+  float* rl = reduction == FLCE_NONE ? static_cast<float*>(loss->data)
+              : (opt && opt->row_loss) ? opt->row_loss : reinterpret_cast<float*>(b + off_rl);
+  const float* row_grad = opt ? opt->row_grad : nullptr;
   float* lse = (opt && opt->lse) ? opt->lse : reinterpret_cast<float*>(b + off_lse);
   float* zt = reinterpret_cast<float*>(b + off_zt);
   float* pm = reinterpret_cast<float*>(b + off_pm);
@@ -736,7 +759,8 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   if (st != FLCE_OK) return st;
   for (int64_t r0 = 0; r0 < BT; r0 += 65535 * 32) {
     const int rows = (int)std::min<int64_t>(65535 * 32, BT - r0);
-    CombineArgs a{tgt + r0, ignore_index, V, rows, (int)ntile, ldp, pm + r0, ps + r0, zt + r0, rl + r0, lse + r0, nv, reduction};
+    CombineArgs a{tgt + r0, ignore_index, V, rows, (int)ntile, ldp, pm + r0, ps + r0, zt + r0, rl + r0, lse + r0, nv, reduction,
+                  row_grad ? row_grad + r0 : nullptr};
     st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
     if (st != FLCE_OK) return st;
   }
@@ -747,17 +771,20 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
       if (dt == FLCE_BF16) {
         CeGradArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
                                     static_cast<__nv_bfloat16*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
-                                    tgt + r0, ignore_index, V, lse + r0, nv, reduction};
+                                    tgt + r0, ignore_index, V, lse + r0, nv, reduction,
+                                    row_grad ? row_grad + r0 : nullptr};
         st = L.run(3, [&] { ce_grad_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a); });
       } else {
         CeGradArgs<float> a{static_cast<const float*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
                             static_cast<float*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
-                            tgt + r0, ignore_index, V, lse + r0, nv, reduction};
+                            tgt + r0, ignore_index, V, lse + r0, nv, reduction,
+                            row_grad ? row_grad + r0 : nullptr};
         st = L.run(3, [&] { ce_grad_kernel<float><<<grid, 256, 0, stream>>>(a); });
       }
       if (st != FLCE_OK) return st;
     }
   }
+  if (reduction == FLCE_NONE) return FLCE_OK;
   return L.run(5, [&] {
     finalize_loss_kernel<<<1, 1024, 0, stream>>>(rl, BT, nv, reduction, static_cast<float*>(loss->data));
   });

@@ -24,6 +24,9 @@ The call shape follows the low-level API of "Liger-Kernel 項目詳細介紹"
 
 Readings where the pages are silent (each also listed in the design doc):
   * mean divides by N, the count of non-ignored rows;
+  * 'none' returns the per-row losses (0 for ignored rows), as the torch loss
+    modules the pages' low-level API mirrors do; with an upstream gradient
+    per row, each dlogits row is scaled by it;
   * N = 0 (every row ignored) gives loss 0 and zero gradients, not NaN;
   * a target outside [0, V) that is not ignore_index is an error (ValueError);
   * a row whose target equals ignore_index is ignored even if ignore_index is
@@ -94,7 +97,7 @@ def row_logsumexp(z: np.ndarray) -> np.ndarray:
 def _scale(reduction: str, n_valid: int) -> float:
     if reduction == "mean":
         return 0.0 if n_valid == 0 else 1.0 / n_valid
-    if reduction == "sum":
+    if reduction in ("sum", "none"):
         return 1.0
     raise ValueError(f"unknown reduction {reduction!r}")
 
@@ -141,11 +144,14 @@ def dlogits(z: np.ndarray, target: np.ndarray, ignore_index: int = -100,
 
 def flce(X, W, target, ignore_index: int = -100, reduction: str = "mean",
          n_valid: Optional[int] = None, want_grad_X: bool = True,
-         want_grad_W: bool = True, block_rows: int = 4096) -> dict:
+         want_grad_W: bool = True, block_rows: int = 4096, row_grad=None) -> dict:
     """Loss, per-row losses, lse and both gradients of FLCE in float64.
 
-    Returns a dict with keys loss (float), row_loss [BT], lse [BT], n_valid,
-    grad_X [BT,H] (or None) and grad_W [V,H] (or None).
+    reduction 'none' returns the per-row losses as `loss`. row_grad [BT]
+    (default all ones) is an upstream gradient per row: the gradients are
+    those of sum_i row_grad_i * l_i * s, s = 1/N (mean) or 1 (sum, none).
+    Returns a dict with keys loss (float, or [BT] for 'none'), row_loss [BT],
+    lse [BT], n_valid, grad_X [BT,H] (or None) and grad_W [V,H] (or None).
     """
     X = _f64(X)
     W = _f64(W)
@@ -155,6 +161,7 @@ def flce(X, W, target, ignore_index: int = -100, reduction: str = "mean",
     valid = valid_mask(target, V, ignore_index)
     N = int(valid.sum()) if n_valid is None else int(n_valid)
     s = _scale(reduction, N)
+    g = np.ones(BT) if row_grad is None else _f64(row_grad).reshape(BT)
 
     row_loss = np.zeros(BT)
     lse = np.zeros(BT)
@@ -169,13 +176,16 @@ def flce(X, W, target, ignore_index: int = -100, reduction: str = "mean",
         tb = target[r0:r1]
         rows = np.nonzero(vb)[0]
         row_loss[r0 + rows] = lse_b[rows] - _target_logits(z, rows, tb)
-        dz = _softmax_minus_onehot(z, lse_b, tb, vb, s)
+        dz = _softmax_minus_onehot(z, lse_b, tb, vb, s) * g[r0:r1, None]
         if want_grad_X:
             grad_X[r0:r1] = _grad_X(dz, W)
         if want_grad_W:
             grad_W += _grad_W(dz, X[r0:r1])
     total = float(row_loss.sum())
-    loss = total * s if reduction == "mean" else total
+    if reduction == "none":
+        loss = row_loss.copy()
+    else:
+        loss = total * s if reduction == "mean" else total
     return {"loss": loss, "row_loss": row_loss, "lse": lse, "n_valid": N,
             "grad_X": grad_X, "grad_W": grad_W}
 

@@ -215,3 +215,51 @@ def test_host_buffers_end_to_end():
     ref = oracle.flce(d["X"], d["W"], d["target"])
     assert rel_err(loss.item(), ref["loss"]) <= 1e-3
     assert_grad_close(gW, ref["grad_W"], "bf16", "grad_W")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_none_reduction_with_row_grad(dtype):
+    w = WORKLOADS["tiny"] if dtype == "f32" else WORKLOADS["llama3_8b_seq"]
+    d = make_inputs(w, BT=300, H=128, V=2000)
+    g = np.random.default_rng(3).standard_normal(300).astype(np.float32)
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, reduction="none", row_grad=torch.from_numpy(g).cuda(),
+                                                  chunk_rows=128)
+    torch.cuda.synchronize()
+    ref = oracle.flce(d["X"], d["W"], d["target"], reduction="none", row_grad=g)
+    assert loss.shape == (300,)
+    np.testing.assert_allclose(loss.cpu().numpy(), ref["loss"], rtol=TOL[dtype]["loss"], atol=TOL[dtype]["loss"])
+    assert_grad_close(gX, ref["grad_X"], dtype, "grad_X (none)")
+    assert_grad_close(gW, ref["grad_W"], dtype, "grad_W (none)")
+
+
+def test_cross_entropy_none_reduction():
+    rng = np.random.default_rng(8)
+    BT, V = 200, 3000
+    z = torch.from_numpy((rng.standard_normal((BT, V)) * 2).astype(np.float32)).to(torch.bfloat16)
+    t = rng.integers(0, V, BT)
+    t[::9] = IGNORE_INDEX
+    g = rng.standard_normal(BT).astype(np.float32)
+    z64 = z.double().numpy()
+    ref_rows = oracle.cross_entropy(z64, t, reduction="none")["row_loss"]
+    ref_dz = oracle.dlogits(z64, t, reduction="sum") * g[:, None]
+    loss, dz = L().cross_entropy(z.cuda(), torch.from_numpy(t).cuda(), reduction="none",
+                                 row_grad=torch.from_numpy(g).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(loss.cpu().numpy(), ref_rows, rtol=1e-3, atol=1e-3)
+    assert_grad_close(dz, ref_dz, "bf16", "dz (none)")
+
+
+def test_module_none_reduction_backward():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
+    X, W, t = to_dev(d)
+    X = X.reshape(2, 128, 128).clone().requires_grad_(True)
+    W = W.clone().requires_grad_(True)
+    rows = L().FusedLinearCrossEntropyLoss(reduction="none")(W, X, t.reshape(2, 128))
+    assert rows.shape == (2, 128)
+    g = torch.randn(2, 128, device="cuda", generator=torch.Generator(device="cuda").manual_seed(1))
+    rows.backward(g)
+    ref = oracle.flce(d["X"], d["W"], d["target"], reduction="none", row_grad=g.reshape(-1).cpu().numpy())
+    np.testing.assert_allclose(rows.detach().reshape(-1).cpu().numpy(), ref["loss"], rtol=1e-3, atol=1e-3)
+    assert_grad_close(X.grad.reshape(256, 128), ref["grad_X"], "bf16", "module grad_X (none)")
+    assert_grad_close(W.grad, ref["grad_W"], "bf16", "module grad_W (none)")

@@ -390,3 +390,25 @@ def test_golden_tiny_regression():
         np.testing.assert_allclose(r["grad_W"][:4, :8], g[red]["grad_W_rows0to3_first8"], rtol=1e-9, atol=1e-18)
     # loss of a near-uniform softmax over 4096 classes sits near ln 4096
     assert abs(g["mean"]["loss"] - math.log(4096)) < 0.3
+
+
+def test_none_reduction_and_row_grad_against_torch():
+    """reduction 'none' with an upstream gradient per row: torch float64 autograd."""
+    X, W, t = _rand_case(BT=11, H=5, V=9, ignore=(2, 7), seed=21)
+    g = np.random.default_rng(5).standard_normal(11)
+    r = oracle.flce(X, W, t, reduction="none", row_grad=g)
+    Xt = torch.tensor(X, requires_grad=True)
+    Wt = torch.tensor(W, requires_grad=True)
+    rows = torch.nn.functional.cross_entropy(Xt @ Wt.T, torch.tensor(t), ignore_index=IGNORE_INDEX,
+                                             reduction="none")
+    rows.backward(torch.tensor(g))
+    np.testing.assert_allclose(r["loss"], rows.detach().numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(r["grad_X"], Xt.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(r["grad_W"], Wt.grad.numpy(), rtol=1e-10, atol=1e-14)
+    # weights of 1 give back the 'sum' gradients; weights 1/N the 'mean' ones
+    s = oracle.flce(X, W, t, reduction="sum")
+    n1 = oracle.flce(X, W, t, reduction="none", row_grad=np.ones(11))
+    np.testing.assert_allclose(n1["grad_W"], s["grad_W"], atol=1e-15)
+    m = oracle.flce(X, W, t, reduction="mean")
+    nm = oracle.flce(X, W, t, reduction="sum", row_grad=np.full(11, 1.0 / m["n_valid"]))
+    np.testing.assert_allclose(nm["grad_X"], m["grad_X"], atol=1e-15)
