@@ -205,7 +205,6 @@ FLCE_API flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const
                                                 flce_tensor* grad_logits, flce_stream_t stream);
 
 /*
- * Plain bf16 GEMM on the library's tcgen05 engine,/*
  * Plain bf16 GEMM on the library's tcgen05 engine, for testing that engine
  * on its own: C[M,N] (f32, row-major, ldc) = sum_k A(m,k) * B(n,k).
  * A is [M,K] row-major (a_mn_major = 0, lda >= K) or [K,M] row-major

@@ -158,3 +158,22 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(B, "LIB_PATH", "/nonexistent/libflce.so")
     with pytest.raises(RuntimeError, match="not built"):
         B.lib()
+
+
+def test_plain_c_caller(tmp_path, lib):
+    """The ABI works from C: compile tests/c/abi_smoke.c against include/flce.h."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_smoke"
+    libdir = os.path.dirname(B.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "abi_smoke.c"), "-o", str(exe),
+                        "-L", libdir, "-l:libflce.so", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.strip().endswith("ok")
