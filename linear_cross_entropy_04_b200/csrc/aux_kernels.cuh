@@ -225,6 +225,9 @@ struct CePartialArgs {
 
 template <typename T>
 __global__ void __launch_bounds__(256) ce_partials_kernel(CePartialArgs<T> a) {
+  // One warp per (row, tile of 1024 columns): each lane holds 32 values in
+  // registers, read once as four 16-byte vectors when the tile is whole and
+  // aligned (bf16), so the tile's max and sum-exp cost one pass over memory.
   const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t r = warp_global / a.ntile;
@@ -233,12 +236,29 @@ __global__ void __launch_bounds__(256) ce_partials_kernel(CePartialArgs<T> a) {
   const int64_t n0 = (int64_t)j << a.tile_shift;
   const int64_t n1 = (n0 + (1 << a.tile_shift)) < a.V ? (n0 + (1 << a.tile_shift)) : a.V;
   const T* zr = a.z + r * a.ldz;
-  float m = -INFINITY;
-  for (int64_t c = n0 + lane; c < n1; c += 32) m = fmaxf(m, Vec8<T>::ld1(zr + c));
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const float ms = m * LOG2E_F;
-  float s = 0.f;
-  for (int64_t c = n0 + lane; c < n1; c += 32) s += exp2f(fmaf(Vec8<T>::ld1(zr + c), LOG2E_F, -ms));
+  float m = -INFINITY, s = 0.f;
+  const bool vec = sizeof(T) == 2 && a.tile_shift == 10 && n1 - n0 == 1024;
+  if (vec) {
+    float x[32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float f8[8];
+      Vec8<T>::load(zr + n0 + (q * 32 + lane) * 8, f8);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[q * 8 + k] = f8[k];
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) m = fmaxf(m, x[k]);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ms = m * LOG2E_F;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) s += exp2f(fmaf(x[k], LOG2E_F, -ms));
+  } else {
+    for (int64_t c = n0 + lane; c < n1; c += 32) m = fmaxf(m, Vec8<T>::ld1(zr + c));
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ms = m * LOG2E_F;
+    for (int64_t c = n0 + lane; c < n1; c += 32) s += exp2f(fmaf(Vec8<T>::ld1(zr + c), LOG2E_F, -ms));
+  }
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) {
     a.part_m[(int64_t)j * a.ldp + r] = m;

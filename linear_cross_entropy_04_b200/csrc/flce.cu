@@ -517,7 +517,10 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         prm.prob[0] = make_problem(eg, rows, (int)V, (int)H, 0, 0, EPI_LOGITS, 1);
         prm.lg = LogitsArgs{tgt_c, ignore_index, V, E, pl.lde, pm, ps, pl.ldp, zt};
         prm.err = dev->err;
-        st = L.run(1, [&] { launch_tc(eg, ta, tb, z, z, prm, dev, stream); });
+        // the pair engine writes the chunk store through TMA boxes
+        CUtensorMap te;
+        if (!make_out_tmap(&te, E, rows, V, pl.lde)) return FLCE_ERR_CUDA;
+        st = L.run(1, [&] { launch_tc(eg, ta, tb, z, z, prm, dev, stream, &te); });
         if (st != FLCE_OK) return st;
       }
     } else {

@@ -93,6 +93,80 @@ __device__ __forceinline__ void epi_bf16_tma(const CUtensorMap* tmC, bool store,
   }
 }
 
+// Logits epilogue of the pair engine: as epi_logits (tile max, then e = exp(z - max),
+// its sum and the target logit per row), but the bf16 e tile leaves through
+// shared memory and TMA stores instead of per-row global stores.
+template <typename Release>
+__device__ __forceinline__ void epi_logits_tma(const TcParams& p, const TcProblem& P, const CUtensorMap* tmE,
+                                               int64_t r_base, int q, int tn, int row, uint32_t taddr,
+                                               uint8_t* boxes, uint32_t& issued, const Release& release) {
+  const LogitsArgs& g = p.lg;
+  const int lane = threadIdx.x & 31;
+  const int64_t r = r_base + row;
+  const int64_t rwarp = r_base + q * 32;
+  const bool row_ok = r < P.M;
+  const int64_t n0 = (int64_t)tn * TC_BN;
+  const int ncols = (int)((g.V - n0) < TC_BN ? (g.V - n0) : TC_BN);
+  int tcol = -1;
+  if (row_ok) {
+    const int64_t t = g.target[r];
+    if (t != g.ignore_index && t >= n0 && t < n0 + ncols) tcol = (int)(t - n0);
+  }
+  uint32_t v[32];
+  float mx = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < TC_BN / 32; ++c) {
+    __syncwarp();
+    tmem_ld_32x32(taddr + c * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (c * 32 + j < ncols) mx = fmaxf(mx, __uint_as_float(v[j]));
+  }
+  const float ms = mx * LOG2E_F;
+  float s = 0.f, ztv = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < TC_BN / 32; ++c) {
+    __syncwarp();
+    tmem_ld_32x32(taddr + c * 32, v);
+    tmem_ld_wait();
+    if (c == TC_BN / 32 - 1) release();
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const int col = c * 32 + j;
+      const float z0 = __uint_as_float(v[j]), z1 = __uint_as_float(v[j + 1]);
+      const float e0 = col < ncols ? exp2f(fmaf(z0, LOG2E_F, -ms)) : 0.f;
+      const float e1 = col + 1 < ncols ? exp2f(fmaf(z1, LOG2E_F, -ms)) : 0.f;
+      s += e0 + e1;
+      if (col == tcol) ztv = z0;
+      if (col + 1 == tcol) ztv = z1;
+      pk[j / 2] = pack_bf16x2(e0, e1);
+    }
+    if (rwarp >= P.M || c * 32 >= ncols) continue;  // box wholly outside: warp-uniform
+    uint8_t* box = boxes + (issued & 1) * T2_STAGE_OUT_BYTES;
+    if (issued >= 2) {
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+    }
+    uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmE, box, (int32_t)(n0 + c * 32), (int32_t)rwarp);
+      bulk_commit_group();
+    }
+    ++issued;
+  }
+  if (row_ok) {
+    g.part_m[(int64_t)tn * g.ldp + r] = mx;
+    g.part_s[(int64_t)tn * g.ldp + r] = s;
+    if (tcol >= 0) g.zt[r] = ztv;
+  }
+}
+
 struct ReleasePair {  // 2-CTA engine: one arrival per epilogue warp on the leader's barrier
   uint32_t leader_bar;  // shared::cluster address
   __device__ __forceinline__ void operator()() const {
@@ -282,7 +356,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       const bool tma_out = P.epi == EPI_STORE_BF16 ||
                            (P.epi == EPI_GRADW && (P.gw_mode == GW_STORE_BF16 || P.gw_mode == GW_ADD_BF16));
       if (P.epi == EPI_LOGITS)
-        epi_logits(p, P, r_base, tn, row, taddr, rel);
+        epi_logits_tma(p, P, &tmC0, r_base, q, tn, row, taddr, my_boxes, issued, rel);
       else if (tma_out)
         epi_bf16_tma(T.prob == 0 ? &tmC0 : &tmC1, P.epi == EPI_STORE_BF16 || P.gw_mode == GW_STORE_BF16, P.M, P.N,
                      r_base + q * 32, tn, taddr, my_boxes, issued, rel);

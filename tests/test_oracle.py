@@ -412,3 +412,113 @@ def test_none_reduction_and_row_grad_against_torch():
     m = oracle.flce(X, W, t, reduction="mean")
     nm = oracle.flce(X, W, t, reduction="sum", row_grad=np.full(11, 1.0 / m["n_valid"]))
     np.testing.assert_allclose(nm["grad_X"], m["grad_X"], atol=1e-15)
+
+
+# ------------------------------------------------------------ preference losses
+
+from oracle import preference_oracle as po  # noqa: E402
+
+PREF = ["dpo", "orpo", "cpo", "simpo", "kto"]
+
+
+def _pref_case(seed=0, B=2, T=4, H=3, V=6):
+    rng = np.random.default_rng(seed)
+    N = 2 * B
+    X = rng.standard_normal((N * T, H))
+    W = rng.standard_normal((V, H)) * 0.7
+    t = rng.integers(0, V, (N, T))
+    t[:, 0] = IGNORE_INDEX  # a prompt position in every sequence
+    t[1, 3] = IGNORE_INDEX  # padding
+    kw = {}
+    return X, W, t, kw
+
+
+def _pref_kw(kind, N, rng):
+    if kind == "dpo":
+        return {"ref_logps": rng.standard_normal(N)}
+    if kind == "kto":
+        return {"ref_logps": rng.standard_normal(N), "desirable": np.array([1, 0, 1, 1])}
+    return {}
+
+
+@pytest.mark.parametrize("kind", PREF)
+def test_preference_finite_differences(kind):
+    X, W, t, _ = _pref_case()
+    kw = _pref_kw(kind, 4, np.random.default_rng(1))
+    r = po.preference(kind, X, W, t, beta=0.7, **kw)
+    h = 1e-6
+    for M, g in ((X, r["grad_X"]), (W, r["grad_W"])):
+        num = np.zeros_like(M)
+        for idx in np.ndindex(*M.shape):
+            Mp, Mm = M.copy(), M.copy()
+            Mp[idx] += h
+            Mm[idx] -= h
+            args_p = (Mp, W) if M is X else (X, Mp)
+            args_m = (Mm, W) if M is X else (X, Mm)
+            lp = po.preference(kind, *args_p, t, beta=0.7, **kw)["loss"]
+            lm = po.preference(kind, *args_m, t, beta=0.7, **kw)["loss"]
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-5, atol=1e-9)
+
+
+def test_preference_closed_forms_for_identical_pairs():
+    """Chosen == rejected: DPO/CPO pair term = log 2, SimPO = log(1 + e^gamma),
+    ORPO = NLL + lam * log 2, KTO at r = z0 = 0.5."""
+    X, W, t, _ = _pref_case(seed=3)
+    N, T = t.shape
+    B = N // 2
+    X = X.reshape(N, T, -1)
+    X[B:] = X[:B]
+    t[B:] = t[:B]
+    X = X.reshape(N * T, -1)
+    base = oracle.flce(X, W, t.reshape(-1), reduction="none")
+    valid = (t[:B] != IGNORE_INDEX)
+    nll = base["row_loss"].reshape(N, T)[:B][valid].sum() / valid.sum()
+    assert abs(po.preference("dpo", X, W, t)["loss"] - math.log(2)) < 1e-12
+    assert abs(po.preference("cpo", X, W, t)["loss"] - (math.log(2) + nll)) < 1e-12
+    g = 0.3
+    assert abs(po.preference("simpo", X, W, t, gamma=g)["loss"] - math.log1p(math.exp(g))) < 1e-12
+    assert abs(po.preference("orpo", X, W, t, lam=0.25)["loss"] - (nll + 0.25 * math.log(2))) < 1e-12
+    # KTO: with ref = lp every r = 0 = z0, so every term is 1 - sigmoid(0)
+    lp, _, _ = po.sequence_logps(base["row_loss"], t, N)
+    assert abs(po.preference("kto", X, W, t, ref_logps=lp, desirable=np.array([1, 0, 1, 0]))["loss"] - 0.5) < 1e-12
+
+
+@pytest.mark.parametrize("kind", PREF)
+def test_preference_against_torch_float64(kind):
+    X, W, t, _ = _pref_case(seed=5, B=3, T=5, H=4, V=7)
+    rng = np.random.default_rng(2)
+    kw = {"ref_logps": rng.standard_normal(6)} if kind in ("dpo", "kto") else {}
+    if kind == "kto":
+        kw["desirable"] = np.array([1, 1, 0, 1, 0, 0])
+    r = po.preference(kind, X, W, t, beta=0.5, gamma=0.2, lam=0.3, **kw)
+    Xt = torch.tensor(X, requires_grad=True)
+    Wt = torch.tensor(W, requires_grad=True)
+    rows = torch.nn.functional.cross_entropy(Xt @ Wt.T, torch.tensor(t.reshape(-1)), ignore_index=IGNORE_INDEX,
+                                             reduction="none").reshape(6, 5)
+    valid = torch.tensor(t != IGNORE_INDEX, dtype=torch.float64)
+    lp = -(rows * valid).sum(1)
+    c = valid.sum(1)
+    ls = torch.nn.functional.logsigmoid
+    if kind == "kto":
+        rr = lp - torch.tensor(kw["ref_logps"])
+        z0 = torch.clamp(rr.detach().mean(), min=0.0)
+        s = torch.tensor(kw["desirable"], dtype=torch.float64) * 2 - 1
+        L = (1 - torch.sigmoid(0.5 * s * (rr - z0))).mean()
+    else:
+        lw, ll, cw, cl = lp[:3], lp[3:], c[:3], c[3:]
+        nll = (rows[:3] * valid[:3]).sum() / cw.sum()
+        if kind == "dpo":
+            ref = torch.tensor(kw["ref_logps"])
+            L = -ls(0.5 * ((lw - ref[:3]) - (ll - ref[3:]))).mean()
+        elif kind == "cpo":
+            L = -ls(0.5 * (lw - ll)).mean() + nll
+        elif kind == "simpo":
+            L = -ls(0.5 * (lw / cw - ll / cl) - 0.2).mean()
+        else:
+            aw, al = lw / cw, ll / cl
+            L = nll + 0.3 * -ls((aw - torch.log1p(-torch.exp(aw))) - (al - torch.log1p(-torch.exp(al)))).mean()
+    L.backward()
+    assert abs(r["loss"] - L.item()) < 1e-12
+    np.testing.assert_allclose(r["grad_X"], Xt.grad.numpy(), rtol=1e-9, atol=1e-14)
+    np.testing.assert_allclose(r["grad_W"], Wt.grad.numpy(), rtol=1e-9, atol=1e-14)
