@@ -263,3 +263,21 @@ def test_module_none_reduction_backward():
     np.testing.assert_allclose(rows.detach().reshape(-1).cpu().numpy(), ref["loss"], rtol=1e-3, atol=1e-3)
     assert_grad_close(X.grad.reshape(256, 128), ref["grad_X"], "bf16", "module grad_X (none)")
     assert_grad_close(W.grad, ref["grad_W"], "bf16", "module grad_W (none)")
+
+
+def test_host_pipeline_matches_device_call():
+    from linear_cross_entropy_04_b200.pipeline import HostPipeline
+
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=384, H=128, V=1500)
+    X, W, t = to_dev(d)
+    ref = L().fused_linear_cross_entropy(X, W, t)
+    Xh, Wh, th = X.cpu().pin_memory(), W.cpu().pin_memory(), t.cpu().pin_memory()
+    outs = [(torch.empty((), dtype=torch.float32).pin_memory(), torch.empty_like(Xh).pin_memory(),
+             torch.empty_like(Wh).pin_memory()) for _ in range(3)]
+    pipe = HostPipeline(384, 128, 1500)
+    for o in outs:
+        pipe.submit(Xh, Wh, th, o)
+    pipe.synchronize()
+    for o in outs:
+        assert o[0].item() == ref[0].item()
+        assert torch.equal(o[1], ref[1].cpu()) and torch.equal(o[2], ref[2].cpu())
