@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--grad-w-accum", default="output", choices=["output", "fp32"])
+    ap.add_argument("--dp-fused-grad-w", action="store_true",
+                    help="N > 1: reduce-scatter grad_W inside the grad_W GEMM over NVLink (symmetric memory) "
+                         "instead of an NCCL all-reduce after it")
     ap.add_argument("--path", default="flce", choices=["flce", "ce"],
                     help="flce: the fused lm_head + loss step (default); ce: cross-entropy of given logits")
     return ap.parse_args()
@@ -334,7 +337,10 @@ def main():
     from linear_cross_entropy_04_b200.dp import dp_fused_linear_cross_entropy
 
     def step(flags=0):
-        if world > 1:
+        if world > 1 and args.dp_fused_grad_w:
+            # data-parallel step, grad_W reduce-scattered by the grad_W GEMM's epilogue
+            dp_fused_linear_cross_entropy(X, W, t, fused_grad_W=True, flags=flags, **kw)
+        elif world > 1:
             # data-parallel step: all-reduce N before the loss, then loss and grad_W
             dp_fused_linear_cross_entropy(X, W, t, out=(loss, gX, gW), flags=flags, **kw)
         else:
@@ -445,6 +451,8 @@ def main():
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; random-init lm_head weights)",
         "config": {"workload": w.name, "BT": w.BT, "H": w.H, "V": w.V, "global_batch": w.BT * world,
                    "seq_len": w.BT, "parallelism": f"dp{world}",
+                   "grad_w_exchange": ("fused reduce-scatter in the grad_W GEMM" if args.dp_fused_grad_w
+                                       else "NCCL all-reduce") if world > 1 else None,
                    "l2": "inputs larger than L2 (W alone is %.2f GB)" % (w.V * w.H * 2 / 1e9),
                    "chunk_rows": st["chunk_rows"], "n_chunks": st["n_chunks"],
                    "grad_w_accum": args.grad_w_accum},

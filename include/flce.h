@@ -105,6 +105,18 @@ typedef struct {
   const float* row_grad;         /* optional DEVICE [BT] fp32: upstream gradient per row; the
                                     gradients are those of sum_i row_grad_i * l_i * (1/N or 1).
                                     NULL = all ones. */
+  /* grad_W scattered to shards (data parallelism): shard k (< n_shards <= 8) owns grad_W rows
+     [k * shard_rows, (k+1) * shard_rows), stored bf16 [rows, H] with row pitch grad_w_shard_ld
+     at grad_w_shards[k] (a HOST array of device pointers; a shard may live on a peer GPU, mapped
+     into this one). Every grad_W tile is ADDED into its owner's shard as it is produced (a TMA
+     reduce-add, done in the owner's L2, over NVLink for a peer), for every chunk. So the caller
+     zeroes each shard and orders that before any rank's call, and orders every rank's call
+     before reading a shard. Requires the bf16 path, grad_W == NULL, shard_rows % 32 == 0 and
+     n_shards * shard_rows >= V. Additions from several callers land in unspecified order. */
+  void* const* grad_w_shards;
+  int32_t n_shards;
+  int64_t shard_rows;
+  int64_t grad_w_shard_ld;
 } flce_options;
 
 typedef struct {

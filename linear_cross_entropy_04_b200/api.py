@@ -42,7 +42,8 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                chunk_rows: int = 0, workspace_limit_bytes: int = 0,
                                grad_w_accum: str = "output", n_valid: Optional[torch.Tensor] = None,
                                row_loss: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                               row_grad: Optional[torch.Tensor] = None,
+                               row_grad: Optional[torch.Tensor] = None, grad_w_shards=None,
+                               shard_rows: int = 0,
                                flags: int = 0, stream=None, out=None, host_out=None,
                                return_stats: bool = False):
     """Loss, grad_X and grad_W of cross-entropy over X W^T in one call.
@@ -51,6 +52,10 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     reduction 'mean' | 'sum' | 'none' ('none': loss is the [BT] per-row losses).
     row_grad [BT] fp32 scales each row's contribution to the gradients (the
     upstream gradient of the per-row losses); default all ones.
+    grad_w_shards: a list of bf16 [shard_rows, H] tensors (local or mapped
+    from peer GPUs); shard k owns grad_W rows [k*shard_rows, (k+1)*shard_rows)
+    and each grad_W tile is added into its owner shard as it is produced
+    (no grad_W tensor is returned then). The caller zeroes the shards first.
     Tensors on the host are staged to the current CUDA device and the
     results copied back (the end-to-end path); nothing runs on the CPU.
     host_out = (loss, grad_X, grad_W) pinned host tensors receive them then.
@@ -69,13 +74,20 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     else:
         loss = torch.empty((X.shape[0],) if reduction == "none" else (), dtype=torch.float32, device=X.device)
         gX = torch.empty_like(X) if want_grad_X else None
-        gW = torch.empty_like(W) if want_grad_W else None
+        gW = torch.empty_like(W) if want_grad_W and grad_w_shards is None else None
     if row_grad is not None:
         row_grad = row_grad.to(device=X.device, dtype=torch.float32).contiguous()
     o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags, n_valid, row_loss, lse,
                  row_grad=row_grad)
+    if grad_w_shards is not None:
+        shard_ptrs = (ctypes.c_void_p * len(grad_w_shards))(*[t_.data_ptr() for t_ in grad_w_shards])
+        o.grad_w_shards = ctypes.cast(shard_ptrs, ctypes.POINTER(ctypes.c_void_p))
+        o.n_shards = len(grad_w_shards)
+        o.shard_rows = int(shard_rows)
+        o.grad_w_shard_ld = grad_w_shards[0].stride(0)
     st = B.FlceStats()
-    B.check(B.lib().flce_plan(X.shape[0], X.shape[1], W.shape[0], B.dtype_code(X), int(gW is not None),
+    B.check(B.lib().flce_plan(X.shape[0], X.shape[1], W.shape[0], B.dtype_code(X),
+                              int(gW is not None or grad_w_shards is not None),
                               ctypes.byref(o), ctypes.byref(st)), "flce_plan")
     ws = None
     if st.workspace_bytes > 0:

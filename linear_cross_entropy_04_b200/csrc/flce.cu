@@ -76,7 +76,9 @@ flce_status device_ctx(DeviceCtx** out) {
         return FLCE_ERR_CUDA;
       if (cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TC_SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(tc_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(tc_gemm_pair_kernel<NoShards>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               T2_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tc_gemm_pair_kernel<ShardMaps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                T2_SMEM_BYTES) != cudaSuccess)
         return FLCE_ERR_CUDA;
       {
@@ -93,7 +95,7 @@ flce_status device_ctx(DeviceCtx** out) {
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int nc = 0;
-        if (cudaOccupancyMaxActiveClusters(&nc, tc_gemm_pair_kernel, &cfg) != cudaSuccess || nc <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&nc, tc_gemm_pair_kernel<NoShards>, &cfg) != cudaSuccess || nc <= 0) {
           cudaGetLastError();
           nc = c.sms / 2;
         }
@@ -387,16 +389,22 @@ bool make_out_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
 
 void launch_tc(const Engine& eg, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                const CUtensorMap& b1, const TcParams& prm, const DeviceCtx* dev, cudaStream_t stream,
-               const CUtensorMap* c0 = nullptr, const CUtensorMap* c1 = nullptr) {
+               const CUtensorMap* c0 = nullptr, const CUtensorMap* c1 = nullptr, const ShardMaps* shards = nullptr) {
   CUtensorMap zc;
   std::memset(&zc, 0, sizeof(zc));
+  NoShards ns;
+  ns.unused = 0;
   const int sms = dev->sms;
   int64_t tiles = (int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n;
   if (prm.nprob > 1) tiles += (int64_t)prm.prob[1].tiles_m * prm.prob[1].tiles_n;
   if (eg.pair) {
     const int pairs = (int)std::min<int64_t>(dev->pairs, tiles);
-    tc_gemm_pair_kernel<<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(a0, b0, a1, b1, c0 ? *c0 : zc,
-                                                                          c1 ? *c1 : zc, prm);
+    if (shards)
+      tc_gemm_pair_kernel<ShardMaps><<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(
+          a0, b0, a1, b1, c0 ? *c0 : zc, c1 ? *c1 : zc, *shards, prm);
+    else
+      tc_gemm_pair_kernel<NoShards><<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(
+          a0, b0, a1, b1, c0 ? *c0 : zc, c1 ? *c1 : zc, ns, prm);
   } else {
     const int grid = (int)std::min<int64_t>(sms, tiles);
     tc_gemm_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
@@ -433,6 +441,17 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   }
   if (grad_X && (BT > 0 && !check_matrix(grad_X, dt, BT, H))) return FLCE_ERR_INVALID_ARG;
   if (grad_W && !check_matrix(grad_W, dt, V, H)) return FLCE_ERR_INVALID_ARG;
+  // grad_W scattered to (possibly peer) shards
+  const bool sharded = opt && opt->n_shards > 0;
+  if (sharded) {
+    if (dt != FLCE_BF16 || grad_W || !opt->grad_w_shards || opt->n_shards > MAX_SHARDS) return FLCE_ERR_INVALID_ARG;
+    if (opt->shard_rows <= 0 || opt->shard_rows % 32 || opt->shard_rows * opt->n_shards < V) return FLCE_ERR_INVALID_ARG;
+    if (opt->grad_w_shard_ld < H || opt->grad_w_shard_ld % 8 || opt->grad_w_accum != FLCE_GRADW_ACCUM_OUTPUT)
+      return FLCE_ERR_INVALID_ARG;
+    for (int k = 0; k < opt->n_shards; ++k)
+      if (k * opt->shard_rows < V && (!opt->grad_w_shards[k] || !is_aligned(opt->grad_w_shards[k], 16)))
+        return FLCE_ERR_INVALID_ARG;
+  }
   if (dt == FLCE_BF16) {
     // TMA and 16-byte vector stores: 16-byte aligned bases and rows
     if (H % 8 || !is_aligned(W->data, 16) || W->stride[0] % 8) return FLCE_ERR_INVALID_ARG;
@@ -441,7 +460,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     if (grad_W && (!is_aligned(grad_W->data, 16) || grad_W->stride[0] % 8)) return FLCE_ERR_INVALID_ARG;
   }
   const bool want_gx = grad_X != nullptr && BT > 0;
-  const bool want_gw = grad_W != nullptr;
+  const bool want_gw = grad_W != nullptr || sharded;
   const bool need_rowloss = reduction != FLCE_NONE && !(opt && opt->row_loss);
   Plan pl;
   flce_status st = make_plan(BT, H, V, dt, want_gw, opt, need_rowloss, &pl);
@@ -464,8 +483,9 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
 
   if (BT == 0) {
     if (reduction != FLCE_NONE && cudaMemsetAsync(loss->data, 0, 4, stream) != cudaSuccess) return FLCE_ERR_CUDA;
-    if (want_gw && cudaMemset2DAsync(grad_W->data, grad_W->stride[0] * dtype_size(dt), 0,
-                                     H * dtype_size(dt), V, stream) != cudaSuccess)
+    // shards receive additions only: nothing to add for an empty batch
+    if (grad_W && cudaMemset2DAsync(grad_W->data, grad_W->stride[0] * dtype_size(dt), 0,
+                                    H * dtype_size(dt), V, stream) != cudaSuccess)
       return FLCE_ERR_CUDA;
     if (stats) stats->workspace_bytes = 0;
     return FLCE_OK;
@@ -572,6 +592,8 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       CUtensorMap tm[4], tc[2];
       std::memset(tm, 0, sizeof(tm));
       std::memset(tc, 0, sizeof(tc));
+      ShardMaps shard_maps;
+      std::memset(&shard_maps, 0, sizeof(shard_maps));
       TcParams prm;
       std::memset(&prm, 0, sizeof(prm));
       prm.err = dev->err;
@@ -604,11 +626,26 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
             !make_tmap(&tm[2 * np + 1], Xc, H, rows, ldx * 2, 64, 64))
           return FLCE_ERR_CUDA;
         TcProblem P = make_problem(eg, (int)V, (int)H, rows, 1, 1, EPI_GRADW, 0);
-        P.out = grad_W->data;
-        P.ldo = grad_W->stride[0];
-        if (!make_out_tmap(&tc[np], P.out, V, H, grad_W->stride[0])) return FLCE_ERR_CUDA;
+        if (sharded) {
+          if (!eg.pair) return FLCE_ERR_INVALID_ARG;  // shard routing lives in the pair engine's epilogue
+          P.n_shards = opt->n_shards;
+          P.shard_rows = opt->shard_rows;
+          P.gw_mode = GW_ADD_BF16;
+          for (int k = 0; k < opt->n_shards; ++k) {
+            const int64_t r0k = k * opt->shard_rows;
+            if (r0k >= V) break;
+            if (!make_out_tmap(&shard_maps.m[k], opt->grad_w_shards[k], std::min(opt->shard_rows, V - r0k), H,
+                               opt->grad_w_shard_ld))
+              return FLCE_ERR_CUDA;
+          }
+        } else {
+          P.out = grad_W->data;
+          P.ldo = grad_W->stride[0];
+          if (!make_out_tmap(&tc[np], P.out, V, H, grad_W->stride[0])) return FLCE_ERR_CUDA;
+        }
         const bool last = c == pl.n_chunks - 1;
-        if (!pl.facc) P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
+        if (sharded) P.gw_mode = GW_ADD_BF16;
+        else if (!pl.facc) P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
         else P.gw_mode = c == 0 ? GW_STORE_F32 : (last ? GW_FINAL_F32 : GW_ADD_F32);
         P.facc = facc;
         P.ld_facc = H;
@@ -628,10 +665,12 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         std::memset(&z, 0, sizeof(z));
         st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0]); });
         if (st != FLCE_OK) return st;
-        st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1]); });
+        st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1], nullptr,
+                                      sharded ? &shard_maps : nullptr); });
       } else {
         prm.nprob = np;
-        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], &tc[1]); });
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], &tc[1],
+                                      sharded ? &shard_maps : nullptr); });
       }
       if (st != FLCE_OK) return st;
       if (gx_split > 1) {

@@ -66,6 +66,8 @@ struct TcProblem {
   int gw_mode;         // GradWMode (EPI_GRADW)
   float* facc;         // fp32 grad_W accumulator (GW_*_F32 modes)
   int64_t ld_facc;
+  int n_shards;        // EPI_GRADW: > 0 routes each output box to its owner shard (add)
+  int64_t shard_rows;  // rows per shard (multiple of 32)
   int ksplit;          // split-K factor (>= 1): tile t covers K-blocks of split t / (tiles_m*tiles_n)
   int kb_per_split;    // K-blocks per split
   int64_t split_stride;  // elements between the output slices of consecutive splits

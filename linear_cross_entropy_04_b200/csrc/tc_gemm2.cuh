@@ -54,10 +54,24 @@ constexpr int T2_SMEM_BYTES = T2_STAGES * T2_STAGE_BYTES + T2_OUT_BYTES + 1024 +
 // 32 rows in 32-column boxes, alternating two staging boxes, and one lane
 // stores (store = true) or adds (store = false, the add done in L2) each box.
 // Rows and columns outside the tensor map's extent are clipped by the TMA.
+// Output maps of grad_W shards (data parallelism): shard k owns rows
+// [k * shard_rows, (k+1) * shard_rows) and may live on a peer GPU.
+constexpr int MAX_SHARDS = 8;
+struct ShardMaps {
+  CUtensorMap m[MAX_SHARDS];
+};
+// The plain kernel takes this placeholder instead: carrying the 1 KB of shard
+// maps as a kernel parameter measurably slowed every launch (14% per step),
+// so only the sharded instantiation has them.
+struct NoShards {
+  int unused;
+};
+
 template <typename Release>
 __device__ __forceinline__ void epi_bf16_tma(const CUtensorMap* tmC, bool store, int64_t M, int64_t N,
                                              int64_t rwarp, int tn, uint32_t taddr, uint8_t* boxes,
-                                             uint32_t& issued, const Release& release) {
+                                             uint32_t& issued, const Release& release,
+                                             const ShardMaps* shards = nullptr, int64_t shard_rows = 0) {
   const int lane = threadIdx.x & 31;
   const int n0 = tn * 256;
   uint32_t v[32];
@@ -83,10 +97,15 @@ __device__ __forceinline__ void epi_bf16_tma(const CUtensorMap* tmC, bool store,
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      if (store)
+      if (shards) {
+        // the box's 32 rows lie in one shard (shard_rows is a multiple of 32)
+        const int owner = (int)(rwarp / shard_rows);
+        tma_reduce_add_2d(&shards->m[owner], box, n0 + c * 32, (int32_t)(rwarp - owner * shard_rows));
+      } else if (store) {
         tma_store_2d(tmC, box, n0 + c * 32, (int32_t)rwarp);
-      else
+      } else {
         tma_reduce_add_2d(tmC, box, n0 + c * 32, (int32_t)rwarp);
+      }
       bulk_commit_group();
     }
     ++issued;
@@ -176,11 +195,13 @@ struct ReleasePair {  // 2-CTA engine: one arrival per epilogue warp on the lead
   }
 };
 
+template <typename ShardArg>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                         const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
-                        const __grid_constant__ TcParams p) {
+                        const __grid_constant__ ShardArg shard_maps, const __grid_constant__ TcParams p) {
+  constexpr bool kShards = sizeof(ShardArg) == sizeof(ShardMaps);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_u32 + 1023u) & ~1023u) - raw_u32);
@@ -357,6 +378,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                            (P.epi == EPI_GRADW && (P.gw_mode == GW_STORE_BF16 || P.gw_mode == GW_ADD_BF16));
       if (P.epi == EPI_LOGITS)
         epi_logits_tma(p, P, &tmC0, r_base, q, tn, row, taddr, my_boxes, issued, rel);
+      else if (kShards && P.epi == EPI_GRADW && P.n_shards > 0)
+        epi_bf16_tma(nullptr, false, P.M, P.N, r_base + q * 32, tn, taddr, my_boxes, issued, rel,
+                     reinterpret_cast<const ShardMaps*>(&shard_maps), P.shard_rows);
       else if (tma_out)
         epi_bf16_tma(T.prob == 0 ? &tmC0 : &tmC1, P.epi == EPI_STORE_BF16 || P.gw_mode == GW_STORE_BF16, P.M, P.N,
                      r_base + q * 32, tn, taddr, my_boxes, issued, rel);

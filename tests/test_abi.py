@@ -177,3 +177,20 @@ def test_plain_c_caller(tmp_path, lib):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
     assert r.stdout.strip().endswith("ok")
+
+
+def test_grad_W_shard_options_are_validated(lib):
+    X = _t(FAKE, B.BF16, (64, 128))
+    W = _t(FAKE, B.BF16, (1000, 128))
+    tg = _t(FAKE, B.I64, (64,))
+    loss = _t(FAKE, B.F32, ())
+    ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    for rows, n, ld in ((500, 2, 128), (512, 1, 128), (512, 2, 100)):  # rows % 32, n*rows < V, ld < H
+        o = B.FlceOptions()
+        lib.flce_options_init(ctypes.byref(o))
+        o.grad_w_shards = ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p))
+        o.n_shards, o.shard_rows, o.grad_w_shard_ld = n, rows, ld
+        st = B.FlceStats()
+        rc = lib.flce_fwd_bwd_ex(ctypes.byref(X), ctypes.byref(W), ctypes.byref(tg), -100, 0, ctypes.byref(loss),
+                                 None, None, None, ctypes.byref(o), ctypes.byref(st))
+        assert rc == 1, (rows, n, ld)

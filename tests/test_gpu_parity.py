@@ -281,3 +281,22 @@ def test_host_pipeline_matches_device_call():
     for o in outs:
         assert o[0].item() == ref[0].item()
         assert torch.equal(o[1], ref[1].cpu()) and torch.equal(o[2], ref[2].cpu())
+
+
+@pytest.mark.parametrize("n_shards,shard_rows", [(3, 1024), (4, 800)])
+def test_grad_W_shard_routing(n_shards, shard_rows):
+    """grad_W added tile by tile into shards (the data-parallel reduce-scatter path), with every
+    shard on this GPU: shard k must hold rows [k*shard_rows, ...) of the plain grad_W."""
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=700, H=256, V=3000)
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256)
+    shards = [torch.zeros(shard_rows, 256, dtype=torch.bfloat16, device="cuda") for _ in range(n_shards)]
+    loss2, gX2, gW2 = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256, grad_w_shards=shards,
+                                                     shard_rows=shard_rows)
+    torch.cuda.synchronize()
+    assert gW2 is None and loss2.item() == loss.item() and torch.equal(gX2, gX)
+    joined = torch.cat(shards)[:3000]
+    assert torch.equal(joined, gW)  # same adds, same order
+    assert torch.all(torch.cat(shards)[3000:] == 0)
+    ref = oracle.flce(d["X"], d["W"], d["target"])
+    assert_grad_close(joined, ref["grad_W"], "bf16", "sharded grad_W")
