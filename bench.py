@@ -36,7 +36,7 @@ UNIT = "tokens/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama3_8b_seq")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -63,15 +63,19 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    """nvidia-smi clock / throttle samples, kept only where they fall inside
+    the timed region (mark_start / mark_end bracket it on the host clock)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index):
+    def __init__(self, index, period_ms=100):
         self.index = index
+        self.period_ms = period_ms
         self.proc = None
+        self.window = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
 
     def __enter__(self):
@@ -79,11 +83,17 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def mark_start(self):
+        self._t0 = time.time()
+
+    def mark_end(self):
+        self.window = (self._t0, time.time())
 
     def __exit__(self, *a):
         if self.proc:
@@ -94,26 +104,59 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
+    @staticmethod
+    def _stamp(txt):
+        import datetime
+
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(txt, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
+
     def summary(self):
         if not self.proc or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for ln in open(self.path):
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                rows.append((self._stamp(f[0]), float(f[2]), float(f[3]), float(f[4]), f[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+        return self.summarize(rows, self.window, self.period_ms)
+
+    @classmethod
+    def summarize(cls, rows, window, period_ms=100):
+        """rows: (unix time, sm MHz, max MHz, watts, [4 reason fields]). Samples
+        inside the window are used; a window shorter than the sample period
+        takes the samples within one period of it and says so."""
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        scope = "timed region"
+        sel = rows
+        if window is not None and all(r[0] is not None for r in rows):
+            sel = [r for r in rows if window[0] <= r[0] <= window[1]]
+            if not sel:
+                pad = period_ms / 1e3
+                sel = [r for r in rows if window[0] - pad <= r[0] <= window[1] + pad]
+                scope = "within one sample period of the timed region"
+            if not sel:
+                return {"sm_mhz": None, "sm_max_mhz": rows[-1][2], "reasons": ["unsampled"],
+                        "samples": 0, "scope": "no sample near the timed region"}
+        else:
+            scope = "whole run (no timestamps)"
+        reasons = set()
+        for r in sel:
+            for n, v in zip(cls.NAMES, r[4]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        loaded = [s for s in sm if mx and s > 0.3 * mx] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": sel[-1][2],
+                "reasons": sorted(reasons), "samples": len(sel), "power_w": statistics.median(r[3] for r in sel),
+                "scope": scope}
 
 
 # ---------------------------------------------------------------- recorded ncu traffic
@@ -184,12 +227,22 @@ def cpu_model():
     return "unknown"
 
 
+def calibrate_rows(d, Wf, target_s, cap):
+    """Rows whose oracle call takes about target_s: the call has a fixed cost
+    (the [V, H] float64 grad_W it allocates and fills) plus a per-row cost, so
+    both are measured (8 and 40 rows) before extrapolating."""
+    t8 = oracle_sample(d, 8, Wf)
+    t40 = oracle_sample(d, 40, Wf)
+    per_row = max((t40 - t8) / 32, 1e-6)
+    fixed = max(t8 - 8 * per_row, 0.0)
+    return int(max(8, min(cap, (target_s - fixed) / per_row)))
+
+
 def cpu_baseline(d, target_s):
     import numpy as np
 
     Wf = d["W"].astype(np.float64)
-    t = oracle_sample(d, 8, Wf)
-    rows = int(max(8, min(2048, 8 * target_s / max(t, 1e-3))))
+    rows = calibrate_rows(d, Wf, target_s, 4096)
     t = oracle_sample(d, rows, Wf)
     return {"value": rows / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"first {rows} tokens of the workload, full fwd+bwd per token in float64 NumPy "
@@ -208,8 +261,7 @@ def run_reference(args):
     w = WORKLOADS[args.workload]
     d = make_inputs(w)
     Wf = d["W"].astype(np.float64)
-    t1 = oracle_sample(d, 4, Wf)
-    rows = int(max(4, min(1024, 4 * (150.0 / max(1, args.steps + args.warmup)) / max(t1, 1e-3))))
+    rows = calibrate_rows(d, Wf, 150.0 / max(1, args.steps + args.warmup), 4096)
     for _ in range(args.warmup):
         oracle_sample(d, rows, Wf)
     tot = 0.0
@@ -266,14 +318,18 @@ def run_ce(args):
         base = torch.cuda.memory_allocated(dev)
         torch.cuda.reset_peak_memory_stats(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
+        with ClockSampler(0) as clk:
+            time.sleep(0.3)
+            clk.mark_start()
+            e0.record()
+            for _ in range(args.steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            clk.mark_end()
         ms = e0.elapsed_time(e1) / args.steps
         res[name] = {"ms_per_step": ms, "tokens_per_s": w.BT / (ms / 1e3),
-                     "peak_extra_bytes": torch.cuda.max_memory_allocated(dev) - base}
+                     "peak_extra_bytes": torch.cuda.max_memory_allocated(dev) - base, "clocks": clk.summary()}
     # the library's CE workspace (taken from its own pool, invisible to torch's counters):
     # N, per-row loss / lse / target logit, and per-(1024-column tile, row) max and sum-exp
     a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
@@ -288,7 +344,7 @@ def run_ce(args):
             "data": "synthetic", "config": {"workload": f"{w.name} logits", "BT": w.BT, "V": w.V},
             "speedup_vs_torch": res["torch"]["ms_per_step"] / res["ours"]["ms_per_step"],
             "memory_ratio_torch_over_ours": res["torch"]["peak_extra_bytes"] / max(res["ours"]["peak_extra_bytes"], 1),
-            "ours": res["ours"], "torch": res["torch"],
+            "ours": res["ours"], "torch": res["torch"], "clocks": res["ours"]["clocks"],
             "roofline": {"bound": "hbm", "achieved": bytes_moved / (res["ours"]["ms_per_step"] / 1e3) / 1e9,
                          "peak": load_peaks()["hbm_gbs"], "unit": "GB/s",
                          "frac": bytes_moved / (res["ours"]["ms_per_step"] / 1e3) / 1e9 / load_peaks()["hbm_gbs"],
@@ -367,11 +423,13 @@ def main():
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         time.sleep(0.3)
+        clk.mark_start()
         ev0.record(stream)
         for _ in range(args.steps):
             step(flags=B.FLAG_TIME_PHASES)
         ev1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     if world > 1:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)

@@ -1,0 +1,53 @@
+"""Host-side pieces of bench.py: the clock-sample window and the oracle sample sizing."""
+import importlib.util
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+IDLE = ["Not Active"] * 4
+CAP = ["Not Active", "Not Active", "Not Active", "Active"]
+
+
+def test_clock_summary_keeps_only_the_timed_window(bench):
+    rows = [(100.0, 1965, 1965, 150, IDLE), (100.1, 1965, 1965, 150, IDLE),
+            (100.2, 1400, 1965, 990, CAP), (100.3, 1380, 1965, 995, CAP), (100.4, 1390, 1965, 990, CAP),
+            (100.5, 1965, 1965, 200, IDLE)]
+    s = bench.ClockSampler.summarize(rows, (100.15, 100.45))
+    assert s["sm_mhz"] == 1390 and s["samples"] == 3 and s["reasons"] == ["sw_power_cap"]
+    assert s["scope"] == "timed region" and s["sm_max_mhz"] == 1965
+
+
+def test_clock_summary_short_window_and_thermal(bench):
+    hot = ["Active", "Not Active", "Active", "Not Active"]
+    rows = [(10.0, 1965, 1965, 100, IDLE), (10.1, 1200, 1965, 900, hot), (10.9, 1965, 1965, 100, IDLE)]
+    s = bench.ClockSampler.summarize(rows, (10.12, 10.15))  # no sample inside: within one period
+    assert s["samples"] == 1 and s["sm_mhz"] == 1200
+    assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"] and s["scope"].startswith("within")
+    s = bench.ClockSampler.summarize(rows, (20.0, 21.0))
+    assert s["sm_mhz"] is None and s["reasons"] == ["unsampled"]
+    assert bench.ClockSampler.summarize([], None)["reasons"] == ["unsampled"]
+
+
+def test_nvidia_smi_timestamp_parses(bench):
+    t = bench.ClockSampler._stamp("2026/12/02 10:00:00.250")
+    assert t is not None and abs((t % 1) - 0.25) < 1e-6
+    assert bench.ClockSampler._stamp("garbage") is None
+
+
+def test_oracle_sample_sizing_separates_fixed_cost(bench, monkeypatch):
+    # a call costs 1 s fixed + 5 ms per row: 12 s of work is 2200 rows, not 8 * 12 / t(8)
+    monkeypatch.setattr(bench, "oracle_sample", lambda d, n, Wf: 1.0 + 0.005 * n)
+    assert bench.calibrate_rows(None, None, 12.0, 4096) == 2200
+    assert bench.calibrate_rows(None, None, 100.0, 4096) == 4096
+    assert bench.calibrate_rows(None, None, 0.5, 4096) == 8
