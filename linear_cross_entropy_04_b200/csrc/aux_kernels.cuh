@@ -284,35 +284,209 @@ struct CeGradArgs {
   const float* row_grad;  // optional [rows] at row 0
 };
 
+// Each thread handles CEG_VECS 8-element vectors of one row, CEG_SPAN columns
+// apart, issuing all loads before any store (two 16-byte loads in flight per
+// thread keep this pass at copy bandwidth; one per thread is issue-bound).
+constexpr int CEG_VECS = 2;
+constexpr int CEG_SPAN = 256 * 8;
+constexpr int CEG_BLOCK_COLS = CEG_SPAN * CEG_VECS;
+
 template <typename T>
 __global__ void __launch_bounds__(256) ce_grad_kernel(CeGradArgs<T> a) {
   const int64_t r = blockIdx.y;
-  const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (c0 >= a.V) return;
+  const int64_t cb = (int64_t)blockIdx.x * CEG_BLOCK_COLS + threadIdx.x * 8;
   const int64_t t = a.target[r];
   const bool valid = target_valid(t, a.V, a.ignore_index);
   const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
   const float ls = a.lse[r] * LOG2E_F;
-  const T* s = a.z + r * a.ldz + c0;
-  T* d = a.dz + r * a.ldd + c0;
-  const bool full = c0 + 8 <= a.V;
-  float v[8];
-  if (full) {
-    Vec8<T>::load(s, v);
-  } else {
+  const T* s = a.z + r * a.ldz;
+  T* d = a.dz + r * a.ldd;
+  float v[CEG_VECS][8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = c0 + k < a.V ? Vec8<T>::ld1(s + k) : 0.f;
+  for (int i = 0; i < CEG_VECS; ++i) {
+    const int64_t c0 = cb + i * CEG_SPAN;
+    if (c0 >= a.V) continue;
+    if (c0 + 8 <= a.V) {
+      Vec8<T>::load(s + c0, v[i]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[i][k] = c0 + k < a.V ? Vec8<T>::ld1(s + c0 + k) : 0.f;
+    }
   }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float x = valid ? exp2f(fmaf(v[k], LOG2E_F, -ls)) * scale : 0.f;
-    if (valid && c0 + k == t) x -= scale;
-    v[k] = x;
+  for (int i = 0; i < CEG_VECS; ++i) {
+    const int64_t c0 = cb + i * CEG_SPAN;
+    if (c0 >= a.V) continue;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float x = valid ? exp2f(fmaf(v[i][k], LOG2E_F, -ls)) * scale : 0.f;
+      if (valid && c0 + k == t) x -= scale;
+      v[i][k] = x;
+    }
+    if (c0 + 8 <= a.V) {
+      Vec8<T>::store(d + c0, v[i]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (c0 + k < a.V) Vec8<T>::st1(d + c0 + k, v[i][k]);
+    }
   }
-  if (full) {
-    Vec8<T>::store(d, v);
-  } else {
-    for (int k = 0; k < 8 && c0 + k < a.V; ++k) Vec8<T>::st1(d + k, v[k]);
+}
+
+// Logits-given cross-entropy in one read and one write of z (bf16 rows).
+// A thread-block cluster of C CTAs owns one row; CTA k of the cluster holds
+// columns [k * slice, (k + 1) * slice) in registers as packed bf16 pairs
+// (CER_VPT vectors of 8 per thread, all loads issued before any use). Each CTA
+// reduces its slice to (max, sum exp(z - max)); the C pairs are exchanged
+// through distributed shared memory and one cluster barrier, after which every
+// CTA merges them in the same order into the row's lse and writes
+// dz = exp(z - lse) * scale straight from its registers, then subtracts scale
+// at the target column. The merge is the online-softmax combination of the
+// paper review's CrossEntropy kernel with the partial tiles held on chip
+// instead of written out, so z crosses HBM once in and dz once out.
+// 64 registers per thread let 4 CTAs share an SM; exponentials use the PTX
+// ex2.approx.ftz instruction (results below 2^-126 flush to 0).
+constexpr int CER_THREADS = 256;
+constexpr int CER_VPT = 8;                              // 8-element vectors per thread
+constexpr int CER_SLICE = CER_THREADS * CER_VPT * 8;    // max columns per CTA
+constexpr int CER_MAX_CLUSTER = 16;
+#ifndef FLCE_CER_MIN_BLOCKS
+#define FLCE_CER_MIN_BLOCKS 4  // CTAs per SM the register budget is sized for
+#endif
+
+struct CeRowArgs {
+  const __nv_bfloat16* z;
+  int64_t ldz;
+  __nv_bfloat16* dz;      // may be z (in place); null: loss only
+  int64_t ldd;
+  const int64_t* target;  // row 0 of this launch
+  int64_t ignore_index, V;
+  float* row_loss;        // [rows] at row 0: l_i, 0 for ignored rows
+  float* lse_out;         // optional [rows] at row 0
+  const int64_t* n_valid;
+  int reduction;
+  const float* row_grad;  // optional [rows] at row 0
+  int slice;              // columns per CTA: a multiple of 8, at most CER_SLICE
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ float block_reduce_256(float v, bool is_max, float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int o = 16; o > 0; o >>= 1) {
+    const float u = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, u) : v + u;
+  }
+  __syncthreads();  // red[] is free (a previous reduction has been read)
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int k = 1; k < CER_THREADS / 32; ++k) v = is_max ? fmaxf(v, red[k]) : v + red[k];
+  return v;
+}
+
+__global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_cluster_kernel(CeRowArgs a) {
+  __shared__ float red[CER_THREADS / 32];
+  __shared__ float2 parts[CER_MAX_CLUSTER];
+  const uint32_t rank = cluster_ctarank(), csize = cluster_nctarank();
+  const int64_t r = blockIdx.y;
+  // columns fit in 32 bits (V < 2^31 is checked on the host)
+  const int base = (int)rank * a.slice;
+  const int end = base + a.slice < (int)a.V ? base + a.slice : (int)a.V;
+  const __nv_bfloat16* zr = a.z + r * a.ldz;
+  const uint16_t* zbits = reinterpret_cast<const uint16_t*>(zr);
+  const int64_t t64 = a.target[r];
+  const bool valid = target_valid(t64, a.V, a.ignore_index);
+  const int t = valid ? (int)t64 : -1;
+  const bool owns_t = valid && t >= base && t < end;
+  // z_t is read before the cluster barrier, ahead of any in-place store to it
+  const float zt = (threadIdx.x == 0 && owns_t) ? __bfloat162float(zr[t]) : 0.f;
+  constexpr uint32_t NEG_INF_BF16 = 0xff80u;
+  uint32_t w[CER_VPT][4];
+#pragma unroll
+  for (int i = 0; i < CER_VPT; ++i) {
+    const int c = base + ((int)threadIdx.x + i * CER_THREADS) * 8;
+    if (c + 8 <= end) {
+      const uint4 u = *reinterpret_cast<const uint4*>(zr + c);
+      w[i][0] = u.x;
+      w[i][1] = u.y;
+      w[i][2] = u.z;
+      w[i][3] = u.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = c + 2 * q < end ? zbits[c + 2 * q] : NEG_INF_BF16;
+        const uint32_t hi = c + 2 * q + 1 < end ? zbits[c + 2 * q + 1] : NEG_INF_BF16;
+        w[i][q] = lo | (hi << 16);
+      }
+    }
+  }
+  __nv_bfloat162 m2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
+#pragma unroll
+  for (int i = 0; i < CER_VPT; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&w[i][q]));
+  float m = fmaxf(__low2float(m2), __high2float(m2));
+  m = block_reduce_256(m, true, red);
+  const float ms = m == -INFINITY ? 0.f : m * LOG2E_F;  // an all -inf slice sums to 0
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < CER_VPT; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      s += ex2_approx(fmaf(bf16_lo(w[i][q]), LOG2E_F, -ms)) + ex2_approx(fmaf(bf16_hi(w[i][q]), LOG2E_F, -ms));
+  s = block_reduce_256(s, false, red);
+  if (threadIdx.x == 0) {
+    const uint32_t slot = smem_u32(&parts[rank]);
+    for (uint32_t q = 0; q < csize; ++q) st_cluster_f32x2(mapa_shared(slot, q), m, s);
+  }
+  cluster_sync();  // every CTA now holds all pairs; no CTA touches a peer after this
+  float M = -INFINITY;
+  for (uint32_t q = 0; q < csize; ++q) M = fmaxf(M, parts[q].x);
+  float S = 0.f;
+  for (uint32_t q = 0; q < csize; ++q)
+    if (parts[q].x != -INFINITY) S += parts[q].y * exp2f((parts[q].x - M) * LOG2E_F);
+  const float lse = M + logf(S);
+  if (threadIdx.x == 0) {
+    if (owns_t) a.row_loss[r] = lse - zt;
+    if (!valid && rank == 0) a.row_loss[r] = 0.f;
+    if (a.lse_out && rank == 0) a.lse_out[r] = lse;
+  }
+  if (!a.dz) return;
+  // 0 for ignored rows: every dz of such a row is exp(.) * 0 = 0
+  const float scale = valid ? mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f) : 0.f;
+  const float ls = lse * LOG2E_F;
+  __nv_bfloat16* dr = a.dz + r * a.ldd;
+#pragma unroll
+  for (int i = 0; i < CER_VPT; ++i) {
+    const int c = base + ((int)threadIdx.x + i * CER_THREADS) * 8;
+    if (c >= end) continue;
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = pack_bf16x2(ex2_approx(fmaf(bf16_lo(w[i][q]), LOG2E_F, -ls)) * scale,
+                         ex2_approx(fmaf(bf16_hi(w[i][q]), LOG2E_F, -ls)) * scale);
+    if (c + 8 <= end) {
+      *reinterpret_cast<uint4*>(dr + c) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      uint16_t* db = reinterpret_cast<uint16_t*>(dr);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (c + 2 * q < end) db[c + 2 * q] = (uint16_t)(o[q] & 0xffffu);
+        if (c + 2 * q + 1 < end) db[c + 2 * q + 1] = (uint16_t)(o[q] >> 16);
+      }
+    }
+  }
+  if (owns_t) {
+    __syncthreads();  // the vector store covering column t comes first
+    if (threadIdx.x == 0) dr[t] = __float2bfloat16_rn(ex2_approx(fmaf(zt, LOG2E_F, -ls)) * scale - scale);
   }
 }
 

@@ -41,6 +41,7 @@ struct DeviceCtx {
   bool supported = false;
   int sms = 0;
   int pairs = 0;  // CTA pairs of the cluster engine that fit on the device at once
+  int ce_max_cluster = 0;  // largest cluster the one-pass cross-entropy kernel can launch with
   uint32_t* err = nullptr;
   cudaMemPool_t pool = nullptr;  // library-owned stream-ordered pool for workspaces
 };
@@ -101,6 +102,27 @@ flce_status device_ctx(DeviceCtx** out) {
         }
         c.pairs = std::min(nc, c.sms / 2);
       }
+      // The one-pass cross-entropy kernel runs clusters of up to 16 CTAs (a
+      // non-portable size) when the device can hold one, else up to 8.
+      c.ce_max_cluster = 8;
+      if (cudaFuncSetAttribute(ce_row_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+          cudaSuccess) {
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = CER_MAX_CLUSTER;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.gridDim = dim3(CER_MAX_CLUSTER, 1, 1);
+        cfg.blockDim = dim3(CER_THREADS);
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int nc = 0;
+        if (cudaOccupancyMaxActiveClusters(&nc, ce_row_cluster_kernel, &cfg) == cudaSuccess && nc > 0)
+          c.ce_max_cluster = CER_MAX_CLUSTER;
+      }
+      cudaGetLastError();
       // A private pool that keeps freed workspace mapped, so repeated calls
       // reuse it stream-ordered instead of mapping and unmapping memory.
       cudaMemPoolProps pp;
@@ -353,6 +375,13 @@ Engine engine() {
 // leave idle. The default picks combined when grad_X alone would keep less
 // than 80% of the workers busy over its waves (measured crossover on B200);
 // FLCE_GRAD_LAUNCH=split|combined forces one.
+// FLCE_CE=multipass selects the partials + combine + grad kernels for bf16
+// logits that the one-pass cluster kernel would otherwise take.
+bool ce_one_pass_enabled() {
+  const char* s = std::getenv("FLCE_CE");
+  return !(s && std::strcmp(s, "multipass") == 0);
+}
+
 bool grad_combined(int64_t gradx_tiles, int64_t units) {
   const char* s = std::getenv("FLCE_GRAD_LAUNCH");
   if (s && std::strcmp(s, "combined") == 0) return true;
@@ -763,12 +792,16 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
     return cudaMemsetAsync(loss->data, 0, 4, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
   }
   const int shift = 10;
-  const int64_t ntile = ceil_div(V, 1 << shift), ldp = round_up(BT, 32);
+  // bf16 rows up to CER_SLICE * (largest cluster) columns take the one-pass
+  // cluster kernel, which needs no partials; the rest take partials + combine + grad
+  const int cer_c = (int)ceil_div(V, CER_SLICE);
+  const bool one_pass = dt == FLCE_BF16 && cer_c <= dev->ce_max_cluster && ce_one_pass_enabled();
+  const int64_t ntile = one_pass ? 0 : ceil_div(V, 1 << shift), ldp = round_up(BT, 32);
   size_t o = 0;
   const size_t off_nv = o; o = align256(o + 8);
   const size_t off_rl = o; o = align256(o + (size_t)BT * 4);
-  const size_t off_lse = o; o = align256(o + (size_t)BT * 4);
-  const size_t off_zt = o; o = align256(o + (size_t)BT * 4);
+  const size_t off_lse = o; o = align256(o + (one_pass ? 0 : (size_t)BT * 4));
+  const size_t off_zt = o; o = align256(o + (one_pass ? 0 : (size_t)BT * 4));
   const size_t off_pm = o; o = align256(o + (size_t)ntile * ldp * 4);
   const size_t off_ps = o; o = align256(o + (size_t)ntile * ldp * 4);
   Workspace ws;
@@ -788,6 +821,36 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   Launcher L{stream, opt && (opt->flags & FLCE_FLAG_TIME_PHASES), env_debug() || (opt && (opt->flags & FLCE_FLAG_SYNC_CHECK))};
   st = L.run(0, [&] { count_valid_kernel<<<1, 1024, 0, stream>>>(tgt, BT, V, ignore_index, nv_local, dev->err); });
   if (st != FLCE_OK) return st;
+  if (one_pass) {
+    const int slice = (int)round_up(ceil_div(V, cer_c), 8);
+    for (int64_t r0 = 0; r0 < BT; r0 += 65535) {
+      const int rows = (int)std::min<int64_t>(65535, BT - r0);
+      CeRowArgs a{static_cast<const __nv_bfloat16*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
+                  grad ? static_cast<__nv_bfloat16*>(grad->data) + r0 * grad->stride[0] : nullptr,
+                  grad ? grad->stride[0] : 0, tgt + r0, ignore_index, V, rl + r0,
+                  (opt && opt->lse) ? opt->lse + r0 : nullptr, nv, reduction, row_grad ? row_grad + r0 : nullptr,
+                  slice};
+      st = L.run(1, [&] {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)cer_c, (unsigned)rows, 1);
+        cfg.blockDim = dim3(CER_THREADS, 1, 1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cer_c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, ce_row_cluster_kernel, a);
+      });
+      if (st != FLCE_OK) return st;
+    }
+    if (reduction == FLCE_NONE) return FLCE_OK;
+    return L.run(5, [&] {
+      finalize_loss_kernel<<<1, 1024, 0, stream>>>(rl, BT, nv, reduction, static_cast<float*>(loss->data));
+    });
+  }
   const int64_t warps = BT * ntile;
   if (dt == FLCE_BF16) {
     CePartialArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data), Z->stride[0], tgt, ignore_index, V,
@@ -809,7 +872,7 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   if (grad) {
     for (int64_t r0 = 0; r0 < BT; r0 += 65535) {
       const int rows = (int)std::min<int64_t>(65535, BT - r0);
-      const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
+      const dim3 grid((unsigned)ceil_div(V, CEG_BLOCK_COLS), (unsigned)rows);
       if (dt == FLCE_BF16) {
         CeGradArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
                                     static_cast<__nv_bfloat16*>(grad->data) + r0 * grad->stride[0], grad->stride[0],
@@ -948,7 +1011,7 @@ flce_status run_ce_noalloc(const flce_tensor* Z, const flce_tensor* target, int6
   if (grad) {
     for (int64_t r0 = 0; r0 < BT; r0 += 65535) {
       const int rows = (int)std::min<int64_t>(65535, BT - r0);
-      const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
+      const dim3 grid((unsigned)ceil_div(V, CEG_BLOCK_COLS), (unsigned)rows);
       if (dt == FLCE_BF16) {
         CeGradArgs<__nv_bfloat16> a{static_cast<const __nv_bfloat16*>(Z->data) + r0 * Z->stride[0], Z->stride[0],
                                     static_cast<__nv_bfloat16*>(grad->data) + r0 * grad->stride[0], grad->stride[0],

@@ -300,3 +300,84 @@ def test_grad_W_shard_routing(n_shards, shard_rows):
     assert torch.all(torch.cat(shards)[3000:] == 0)
     ref = oracle.flce(d["X"], d["W"], d["target"])
     assert_grad_close(joined, ref["grad_W"], "bf16", "sharded grad_W")
+
+
+def _ce_inputs(seed, BT, V, ignore_every=6):
+    rng = np.random.default_rng(seed)
+    z = torch.from_numpy((rng.standard_normal((BT, V)) * 3).astype(np.float32)).to(torch.bfloat16)
+    t = rng.integers(0, V, BT)
+    t[::ignore_every] = IGNORE_INDEX
+    return z, t
+
+
+# V spans one-pass clusters of 1, 2, 4, 8, 10 and 16 CTAs, and a V past the
+# largest cluster (and not a multiple of 8) that takes the multi-pass kernels.
+@pytest.mark.parametrize("V", [1000, 16385, 50000, 128256, 152064, 256000, 300007])
+@pytest.mark.parametrize("mode", ["mean_inplace", "sum", "none_rowgrad", "loss_only"])
+def test_cross_entropy_across_cluster_sizes(V, mode):
+    BT = 48
+    z, t = _ce_inputs(V % 97, BT, V)
+    z64 = z.double().numpy()
+    pitch = V + (-V) % 8
+    buf = torch.zeros(BT, pitch, dtype=torch.bfloat16)
+    buf[:, :V] = z
+    zd = buf.cuda()[:, :V]
+    td = torch.from_numpy(t).cuda()
+    if mode == "none_rowgrad":
+        g = np.random.default_rng(1).standard_normal(BT).astype(np.float32)
+        loss, dz = L().cross_entropy(zd, td, reduction="none", row_grad=torch.from_numpy(g).cuda())
+        ref_rows = oracle.cross_entropy(z64, t, reduction="none")["row_loss"]
+        torch.cuda.synchronize()
+        np.testing.assert_allclose(loss.cpu().numpy(), ref_rows, rtol=1e-3, atol=1e-3)
+        assert_grad_close(dz, oracle.dlogits(z64, t, reduction="sum") * g[:, None], "bf16", "dz (none)")
+        return
+    red = "sum" if mode == "sum" else "mean"
+    lse = torch.full((BT,), float("nan"), dtype=torch.float32, device="cuda")
+    loss, dz = L().cross_entropy(zd, td, reduction=red, inplace=mode == "mean_inplace",
+                                 want_grad=mode != "loss_only", lse=lse)
+    torch.cuda.synchronize()
+    ref = oracle.cross_entropy(z64, t, reduction=red)
+    assert rel_err(loss.item(), ref["loss"]) <= TOL["bf16"]["loss"], (loss.item(), ref["loss"])
+    ref_lse = np.log(np.exp(z64 - z64.max(1, keepdims=True)).sum(1)) + z64.max(1)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=1e-5, atol=1e-4)
+    if mode == "loss_only":
+        assert dz is None
+        return
+    assert_grad_close(dz, ref["dz"], "bf16", f"dz ({mode})")
+    ign = t == IGNORE_INDEX
+    assert torch.all(dz[torch.from_numpy(ign).cuda()] == 0)  # ignored rows exactly 0
+    if mode == "mean_inplace":
+        assert dz.data_ptr() == zd.data_ptr()
+
+
+def test_cross_entropy_one_pass_edge_rows():
+    """All rows ignored (loss 0, dz 0), one row, and -inf logits (masked vocabulary)."""
+    V = 50000
+    z, t = _ce_inputs(3, 5, V)
+    t[:] = IGNORE_INDEX
+    loss, dz = L().cross_entropy(z.cuda(), torch.from_numpy(t).cuda())
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0 and torch.all(dz == 0)
+    z, t = _ce_inputs(4, 1, V)
+    z[0, 20000:40000] = float("-inf")  # two whole CTA slices and parts of others are masked
+    t[0] = 5
+    z64 = z.double().numpy()
+    loss, dz = L().cross_entropy(z.cuda(), torch.from_numpy(t).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.cross_entropy(z64, t)
+    assert np.isfinite(loss.item()) and rel_err(loss.item(), ref["loss"]) <= TOL["bf16"]["loss"]
+    assert torch.all(dz[0, 20000:40000] == 0)
+    assert_grad_close(dz, ref["dz"], "bf16", "dz (-inf)")
+
+
+def test_cross_entropy_one_pass_matches_multipass(monkeypatch):
+    """The one-pass cluster kernel and the partials + combine + grad kernels agree."""
+    z, t = _ce_inputs(9, 256, 128256)
+    zd, td = z.cuda(), torch.from_numpy(t).cuda()
+    l1, g1 = L().cross_entropy(zd, td)
+    monkeypatch.setenv("FLCE_CE", "multipass")
+    l2, g2 = L().cross_entropy(zd, td)
+    torch.cuda.synchronize()
+    assert rel_err(l1.item(), l2.item()) <= 1e-5
+    d = (g1.float() - g2.float()).abs().max().item()
+    assert d <= 2 ** -8 * g2.float().abs().max().item(), d
