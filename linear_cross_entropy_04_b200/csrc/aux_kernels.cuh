@@ -396,16 +396,32 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
   __shared__ float red[CER_THREADS / 32];
   __shared__ float2 parts[CER_MAX_CLUSTER];
   const uint32_t rank = cluster_ctarank(), csize = cluster_nctarank();
-  const int64_t r = blockIdx.y;
+  const int r = blockIdx.y;
   // columns fit in 32 bits (V < 2^31 is checked on the host)
   const int base = (int)rank * a.slice;
   const int end = base + a.slice < (int)a.V ? base + a.slice : (int)a.V;
-  const __nv_bfloat16* zr = a.z + r * a.ldz;
+  const __nv_bfloat16* zr = a.z + (int64_t)r * a.ldz;
   const uint16_t* zbits = reinterpret_cast<const uint16_t*>(zr);
   const int64_t t64 = a.target[r];
   const bool valid = target_valid(t64, a.V, a.ignore_index);
   const int t = valid ? (int)t64 : -1;
   const bool owns_t = valid && t >= base && t < end;
+  if (!valid && !a.lse_out) {
+    // an ignored row needs neither its logits nor a cluster exchange: loss 0,
+    // dz 0 (every CTA of the cluster takes this branch, as they share the row)
+    if (threadIdx.x == 0 && rank == 0) a.row_loss[r] = 0.f;
+    if (a.dz) {
+      __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
+      for (int c = base + (int)threadIdx.x * 8; c < end; c += CER_THREADS * 8) {
+        if (c + 8 <= end) {
+          *reinterpret_cast<uint4*>(dr + c) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          for (int k = c; k < end; ++k) dr[k] = __float2bfloat16_rn(0.f);
+        }
+      }
+    }
+    return;
+  }
   // z_t is read before the cluster barrier, ahead of any in-place store to it
   const float zt = (threadIdx.x == 0 && owns_t) ? __bfloat162float(zr[t]) : 0.f;
   constexpr uint32_t NEG_INF_BF16 = 0xff80u;
@@ -463,7 +479,7 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
   // 0 for ignored rows: every dz of such a row is exp(.) * 0 = 0
   const float scale = valid ? mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f) : 0.f;
   const float ls = lse * LOG2E_F;
-  __nv_bfloat16* dr = a.dz + r * a.ldd;
+  __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
 #pragma unroll
   for (int i = 0; i < CER_VPT; ++i) {
     const int c = base + ((int)threadIdx.x + i * CER_THREADS) * 8;
