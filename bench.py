@@ -48,8 +48,12 @@ def parse():
     ap.add_argument("--dp-fused-grad-w", action="store_true",
                     help="N > 1: reduce-scatter grad_W inside the grad_W GEMM over NVLink (symmetric memory) "
                          "instead of an NCCL all-reduce after it")
-    ap.add_argument("--path", default="flce", choices=["flce", "ce"],
-                    help="flce: the fused lm_head + loss step (default); ce: cross-entropy of given logits")
+    ap.add_argument("--path", default="flce", choices=["flce", "ce", "preference"],
+                    help="flce: the fused lm_head + loss step (default); ce: cross-entropy of given logits; "
+                         "preference: a fused-linear preference loss step (--kind)")
+    ap.add_argument("--kind", default="dpo", choices=["dpo", "orpo", "cpo", "simpo", "kto"],
+                    help="preference loss for --path preference")
+    ap.add_argument("--seq-len", type=int, default=512, help="tokens per sequence for --path preference")
     return ap.parse_args()
 
 
@@ -362,6 +366,107 @@ def run_ce(args):
     return 0
 
 
+# ---------------------------------------------------------------- preference losses
+
+def run_preference(args):
+    """One fused-linear preference-loss step (loss, grad_x, grad_weight) on the
+    lm_head shapes of the workload: its BT tokens form BT / seq_len sequences
+    (chosen rows first, then rejected), the first quarter of each sequence is
+    prompt (ignore_index). Timed against the same loss in plain PyTorch on
+    materialised logits (bf16 matmul, fp32 log-softmax, autograd)."""
+    import numpy as np
+    import torch
+
+    import linear_cross_entropy_04_b200 as flce
+    from linear_cross_entropy_04_b200.inputs import IGNORE_INDEX, WORKLOADS, make_inputs
+    from linear_cross_entropy_04_b200.preference import fused_linear_preference_loss, preference_loss_from_logps
+
+    w = WORKLOADS[args.workload]
+    T = args.seq_len
+    n_seq = w.BT // T
+    assert n_seq >= 2 and n_seq % 2 == 0, "BT / seq_len must be an even number of sequences"
+    d = make_inputs(w, BT=n_seq * T)
+    dev = torch.device("cuda", 0)
+    X = torch.from_numpy(d["X"]).to(torch.bfloat16).to(dev)
+    W = torch.from_numpy(d["W"]).to(torch.bfloat16).to(dev)
+    t = d["target"].reshape(n_seq, T).copy()
+    t[:, : T // 4] = IGNORE_INDEX
+    t = torch.from_numpy(t).to(dev)
+    rng = np.random.default_rng(5)
+    ref = torch.from_numpy(rng.standard_normal(n_seq) * 5.0 - 3000.0).to(dev)
+    des = torch.from_numpy((np.arange(n_seq) % 2).astype(np.float64)).to(dev)
+    kw = dict(ref_logps=ref) if args.kind == "dpo" else dict(desirable=des) if args.kind == "kto" else {}
+
+    def ours():
+        return fused_linear_preference_loss(args.kind, W, X, t, **kw)
+
+    def torch_ref():
+        Xr = X.detach().requires_grad_(True)
+        Wr = W.detach().requires_grad_(True)
+        logits = (Xr @ Wr.t()).float()
+        tt = t.reshape(-1)
+        valid = tt != IGNORE_INDEX
+        lp_tok = torch.log_softmax(logits, -1).gather(1, tt.clamp(min=0)[:, None])[:, 0] * valid
+        row_loss = -lp_tok
+        lp = lp_tok.reshape(n_seq, T).double().sum(1)
+        cnt = valid.reshape(n_seq, T).double().sum(1)
+        nll_sum_chosen = row_loss.reshape(n_seq, T)[: n_seq // 2].double().sum()
+        loss = preference_loss_from_logps(args.kind, lp, cnt, nll_sum_chosen,
+                                          ref_logps=kw.get("ref_logps"), desirable=kw.get("desirable"))
+        loss.backward()
+        return loss, Xr.grad, Wr.grad
+
+    res = {}
+    for name, fn in (("ours", ours), ("torch", torch_ref)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        # peak memory of one step, outputs included, with no earlier step's outputs alive
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        out = fn()
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        loss_val = float(out[0])
+        del out
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(0) as clk:
+            time.sleep(0.3)
+            clk.mark_start()
+            e0.record()
+            for _ in range(args.steps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            clk.mark_end()
+        ms = e0.elapsed_time(e1) / args.steps
+        res[name] = {"ms_per_step": ms, "tokens_per_s": n_seq * T / (ms / 1e3), "peak_extra_bytes": peak,
+                     "loss": loss_val, "clocks": clk.summary()}
+    BT = n_seq * T
+    useful = 6.0 * BT * w.H * w.V
+    peaks = load_peaks()
+    rel = abs(res["ours"]["loss"] - res["torch"]["loss"]) / max(abs(res["torch"]["loss"]), 1e-30)
+    line = {"metric": f"fused-linear {args.kind.upper()} loss fwd+bwd tokens/s", "value": res["ours"]["tokens_per_s"],
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": res["ours"]["ms_per_step"], "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init lm_head weights; prompt quarter of each sequence ignored)",
+            "config": {"workload": f"{w.name} as {n_seq} sequences of {T}", "BT": BT, "H": w.H, "V": w.V,
+                       "kind": args.kind},
+            "speedup_vs_torch": res["torch"]["ms_per_step"] / res["ours"]["ms_per_step"],
+            "memory_ratio_torch_over_ours": res["torch"]["peak_extra_bytes"] / max(res["ours"]["peak_extra_bytes"], 1),
+            "loss_rel_diff_vs_torch": rel, "ours": res["ours"], "torch": res["torch"],
+            "roofline": {"bound": "tensor", "achieved": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12,
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                         "traffic": None, "algorithmic_flops": useful,
+                         "frac_of_burst_peak": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                         "note": "useful 6*BT*H*V; the single-pass schedule executes exactly these, the "
+                                 "two-pass one (batches whose store exceeds the keep budget) 8*BT*H*V"},
+            "clocks": res["ours"]["clocks"]}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def main():
@@ -370,6 +475,8 @@ def main():
         return run_reference(args)
     if args.path == "ce":
         return run_ce(args)
+    if args.path == "preference":
+        return run_preference(args)
 
     import torch
     import torch.distributed as dist

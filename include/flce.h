@@ -87,6 +87,23 @@ typedef enum {
 
 #define FLCE_FLAG_SYNC_CHECK 0x1  /* synchronise and check for CUDA errors after each launch */
 #define FLCE_FLAG_TIME_PHASES 0x2 /* record CUDA events around each phase (flce_phase_times) */
+/* Two-phase use, for losses whose per-row upstream gradient is known only
+ * after the forward pass (preference losses, reduction 'none' under autograd):
+ *   KEEP_LOGITS: forward only. The whole batch is one chunk (BT <= 32768);
+ *     its store of exp(z - m_tile), the per-tile maxima and the row lse stay in
+ *     the caller's workspace (opt->workspace, sized by flce_plan with the same
+ *     options). loss (and row_loss / lse) are written; grad_X and grad_W must
+ *     be NULL.
+ *   FROM_KEPT: gradients only, from what a KEEP_LOGITS call with the same X, W,
+ *     target, ignore_index and workspace left there, with opt->row_grad and the
+ *     reduction's scale applied now; the logits GEMM is not run again. loss is
+ *     not written. Nothing may touch the workspace between the two calls.
+ * Together they do 6*BT*H*V tensor FLOPs where a forward call followed by a
+ * full call with row_grad does 8. The paper has no counterpart: its chunked
+ * preference losses take each chunk's gradient in one pass over complete
+ * pairs; keeping the batch's store is the general form of that on one chunk. */
+#define FLCE_FLAG_KEEP_LOGITS 0x4
+#define FLCE_FLAG_FROM_KEPT 0x8
 
 typedef struct {
   int64_t chunk_rows;            /* rows per chunk; 0 = chosen from workspace_limit_bytes.

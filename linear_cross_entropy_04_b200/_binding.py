@@ -18,7 +18,7 @@ LIB_PATH = os.environ.get("FLCE_LIBRARY") or os.path.join(PKG, "libflce.so")
 
 F32, BF16, I64 = 0, 1, 2
 MEAN, SUM, NONE = 0, 1, 2
-FLAG_SYNC_CHECK, FLAG_TIME_PHASES = 0x1, 0x2
+FLAG_SYNC_CHECK, FLAG_TIME_PHASES, FLAG_KEEP_LOGITS, FLAG_FROM_KEPT = 0x1, 0x2, 0x4, 0x8
 GRADW_ACCUM_OUTPUT, GRADW_ACCUM_FP32 = 0, 1
 DEVERR_TARGET_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
 NUM_PHASES = 6

@@ -121,6 +121,74 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     return res + (st.as_dict(),) if return_stats else res
 
 
+class KeptLogits:
+    """What forward_keep leaves for backward_from_kept: the device workspace that
+    holds the batch's store of exp(z - m_tile), its tile maxima and row lse,
+    with the inputs it was computed from. Nothing else may use the workspace
+    until the gradients are taken."""
+
+    def __init__(self, X, W, target, ignore_index, workspace, n_valid):
+        self.X, self.W, self.target = X, W, target
+        self.ignore_index = ignore_index
+        self.workspace = workspace
+        self.n_valid = n_valid
+
+
+def keep_workspace_bytes(BT: int, H: int, V: int, dtype: str = "bf16", want_grad_W: bool = True) -> int:
+    """Workspace a forward_keep / backward_from_kept pair needs (the whole batch as one chunk)."""
+    o = _options(flags=B.FLAG_KEEP_LOGITS)
+    st = B.FlceStats()
+    B.check(B.lib().flce_plan(BT, H, V, B.BF16 if dtype == "bf16" else B.F32, int(want_grad_W),
+                              ctypes.byref(o), ctypes.byref(st)), "flce_plan")
+    return st.workspace_bytes
+
+
+def forward_keep(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor, ignore_index: int = -100,
+                 reduction: str = "mean", n_valid: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, stream=None):
+    """Loss of cross-entropy over X W^T with the batch's chunk store kept for
+    backward_from_kept (FLCE_FLAG_KEEP_LOGITS). Returns (loss, KeptLogits)."""
+    loss = torch.empty((X.shape[0],) if reduction == "none" else (), dtype=torch.float32, device=X.device)
+    o = _options(flags=B.FLAG_KEEP_LOGITS, n_valid=n_valid, lse=lse)
+    st = B.FlceStats()
+    B.check(B.lib().flce_plan(X.shape[0], X.shape[1], W.shape[0], B.dtype_code(X), 1, ctypes.byref(o),
+                              ctypes.byref(st)), "flce_plan")
+    ws = torch.empty(max(st.workspace_bytes, 256), dtype=torch.uint8, device=X.device)
+    o.workspace = ws.data_ptr()
+    o.workspace_bytes = ws.numel()
+    tX, tW, tt, tl = B.tensor(X), B.tensor(W), B.tensor(target), B.tensor(loss)
+    B.check(B.lib().flce_fwd_bwd_ex(ctypes.byref(tX), ctypes.byref(tW), ctypes.byref(tt), int(ignore_index),
+                                    _RED[reduction], ctypes.byref(tl), None, None, B.stream_handle(stream),
+                                    ctypes.byref(o), None), "flce_fwd_bwd_ex (keep)")
+    return loss, KeptLogits(X, W, target, ignore_index, ws, n_valid)
+
+
+def backward_from_kept(kept: KeptLogits, reduction: str = "mean", row_grad: Optional[torch.Tensor] = None,
+                       want_grad_X: bool = True, want_grad_W: bool = True, stream=None):
+    """grad_X, grad_W from a forward_keep (FLCE_FLAG_FROM_KEPT): the gradients
+    of sum_i row_grad_i * l_i * (1/N or 1) without running the logits GEMM again.
+    The kept workspace is released afterwards."""
+    X, W, t = kept.X, kept.W, kept.target
+    if kept.workspace is None:
+        raise RuntimeError("the kept logits were already used")
+    gX = torch.empty_like(X) if want_grad_X else None
+    gW = torch.empty_like(W) if want_grad_W else None
+    if row_grad is not None:
+        row_grad = row_grad.to(device=X.device, dtype=torch.float32).contiguous()
+    o = _options(flags=B.FLAG_FROM_KEPT, n_valid=kept.n_valid, workspace=kept.workspace, row_grad=row_grad)
+    dummy = torch.empty((X.shape[0],) if reduction == "none" else (), dtype=torch.float32, device=X.device)
+    tX, tW, tt, tl = B.tensor(X), B.tensor(W), B.tensor(t), B.tensor(dummy)
+    tgX = B.tensor(gX) if gX is not None else None
+    tgW = B.tensor(gW) if gW is not None else None
+    B.check(B.lib().flce_fwd_bwd_ex(ctypes.byref(tX), ctypes.byref(tW), ctypes.byref(tt), int(kept.ignore_index),
+                                    _RED[reduction], ctypes.byref(tl),
+                                    ctypes.byref(tgX) if tgX is not None else None,
+                                    ctypes.byref(tgW) if tgW is not None else None,
+                                    B.stream_handle(stream), ctypes.byref(o), None), "flce_fwd_bwd_ex (from kept)")
+    kept.workspace = None
+    return gX, gW
+
+
 def cross_entropy(logits: torch.Tensor, target: torch.Tensor, ignore_index: int = -100,
                   reduction: str = "mean", want_grad: bool = True, inplace: bool = False,
                   n_valid: Optional[torch.Tensor] = None, row_loss: Optional[torch.Tensor] = None,
@@ -194,10 +262,12 @@ class _FLCEFunction(torch.autograd.Function):
     once, and backward hands them back scaled by the upstream gradient.
     'none': the forward computes only the per-row losses; backward runs the
     fused path again with the per-row upstream gradient (row_grad), so the
-    logits GEMM is done twice in exchange for never storing dlogits."""
+    logits GEMM is done twice in exchange for never storing dlogits. With
+    keep_logits the forward keeps the batch's bf16 store instead (held until
+    backward) and backward takes the gradients from it."""
 
     @staticmethod
-    def forward(ctx, weight, inp, target, ignore_index, reduction, grad_w_accum):
+    def forward(ctx, weight, inp, target, ignore_index, reduction, grad_w_accum, keep_logits=False):
         shape = inp.shape
         X = inp.reshape(-1, shape[-1])
         if X.stride(-1) != 1 or (X.stride(0) % 8 and X.dtype == torch.bfloat16):
@@ -208,10 +278,14 @@ class _FLCEFunction(torch.autograd.Function):
         ctx.ignore_index = ignore_index
         ctx.grad_w_accum = grad_w_accum
         if reduction == "none":
+            ctx.need = (ctx.needs_input_grad[1], ctx.needs_input_grad[0])
+            ctx.kept = None
+            if keep_logits:
+                loss, ctx.kept = forward_keep(X, weight, t, ignore_index=ignore_index, reduction="none")
+                return loss.reshape(shape[:-1])
             loss, _, _ = fused_linear_cross_entropy(X, weight, t, ignore_index=ignore_index, reduction="none",
                                                     want_grad_X=False, want_grad_W=False)
             ctx.save_for_backward(X, weight, t)
-            ctx.need = (ctx.needs_input_grad[1], ctx.needs_input_grad[0])
             return loss.reshape(shape[:-1])
         loss, gX, gW = fused_linear_cross_entropy(
             X, weight, t, ignore_index=ignore_index, reduction=reduction,
@@ -224,34 +298,44 @@ class _FLCEFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, grad_out):
         if ctx.reduction == "none":
-            X, W, t = ctx.saved_tensors
             want_x, want_w = ctx.need
-            _, gX, gW = fused_linear_cross_entropy(X, W, t, ignore_index=ctx.ignore_index, reduction="none",
-                                                   row_grad=grad_out.reshape(-1), want_grad_X=want_x,
-                                                   want_grad_W=want_w, grad_w_accum=ctx.grad_w_accum)
-            return gW, (gX.reshape(ctx.shape) if gX is not None else None), None, None, None, None
+            if ctx.kept is not None:
+                gX, gW = backward_from_kept(ctx.kept, reduction="none", row_grad=grad_out.reshape(-1),
+                                            want_grad_X=want_x, want_grad_W=want_w)
+                ctx.kept = None
+            else:
+                X, W, t = ctx.saved_tensors
+                _, gX, gW = fused_linear_cross_entropy(X, W, t, ignore_index=ctx.ignore_index, reduction="none",
+                                                       row_grad=grad_out.reshape(-1), want_grad_X=want_x,
+                                                       want_grad_W=want_w, grad_w_accum=ctx.grad_w_accum)
+            return gW, (gX.reshape(ctx.shape) if gX is not None else None), None, None, None, None, None
         gX, gW = ctx.saved_tensors
         hx, hw = ctx.has
         one = grad_out.numel() == 1 and bool(grad_out == 1)
         dX = (gX if one else gX * grad_out.to(gX.dtype)).reshape(ctx.shape) if hx else None
         dW = (gW if one else gW * grad_out.to(gW.dtype)) if hw else None
-        return dW, dX, None, None, None, None
+        return dW, dX, None, None, None, None, None
 
 
 class FusedLinearCrossEntropyLoss(torch.nn.Module):
     """loss_fn(lm_head.weight, input, target) -> scalar loss with autograd.
 
     input may be [BT, H] or [B, T, H]; target has the matching leading shape.
-    reduction 'none' returns the per-row losses with the leading shape.
+    reduction 'none' returns the per-row losses with the leading shape; with
+    keep_logits=True its forward keeps the batch's bf16 store until backward
+    (BT * V * 2 bytes held, 6 rather than 8 * BT * H * V tensor FLOPs).
     """
 
-    def __init__(self, ignore_index: int = -100, reduction: str = "mean", grad_w_accum: str = "output"):
+    def __init__(self, ignore_index: int = -100, reduction: str = "mean", grad_w_accum: str = "output",
+                 keep_logits: bool = False):
         super().__init__()
         if reduction not in _RED:
             raise ValueError("reduction must be 'mean', 'sum' or 'none'")
         self.ignore_index = ignore_index
         self.reduction = reduction
         self.grad_w_accum = grad_w_accum
+        self.keep_logits = keep_logits
 
     def forward(self, weight, input, target):  # noqa: A002 - mirrors the pages' call
-        return _FLCEFunction.apply(weight, input, target, self.ignore_index, self.reduction, self.grad_w_accum)
+        return _FLCEFunction.apply(weight, input, target, self.ignore_index, self.reduction, self.grad_w_accum,
+                                   self.keep_logits)

@@ -73,6 +73,7 @@ struct CombineArgs {
   const int64_t* n_valid;
   int reduction;
   const float* row_grad;  // optional [rows] at chunk row 0: upstream gradient per row
+  int skip_factors;       // 1: leave the tile maxima in part_m (factor_kernel turns them later)
 };
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     }
   }
   __syncthreads();
-  if (row_ok) {
+  if (row_ok && !a.skip_factors) {
     const bool valid = target_valid(a.target[r], a.V, a.ignore_index);
     const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
     const float lse = sm_lse[lane];
@@ -120,6 +121,33 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       float* pm = a.part_m + (int64_t)j * a.ldp + r;
       *pm = valid ? exp2f((*pm - lse) * LOG2E_F) * scale : 0.f;
     }
+  }
+}
+
+// The factor step of combine_kernel on its own, for gradients taken from a
+// kept forward pass: part_m holds the tile maxima, lse the row lse.
+struct FactorArgs {
+  const int64_t* target;  // chunk row 0
+  int64_t ignore_index, V;
+  int rows, ntile;
+  int64_t ldp;
+  float* part_m;          // in: tile max; out: exp(m_tile - lse) * scale (0 for ignored rows)
+  const float* lse;       // [rows]
+  const int64_t* n_valid;
+  int reduction;
+  const float* row_grad;  // optional [rows]
+};
+
+__global__ void __launch_bounds__(256) factor_kernel(FactorArgs a) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int r = blockIdx.x * 32 + lane;
+  if (r >= a.rows) return;
+  const bool valid = target_valid(a.target[r], a.V, a.ignore_index);
+  const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
+  const float lse = a.lse[r];
+  for (int j = w; j < a.ntile; j += 8) {
+    float* pm = a.part_m + (int64_t)j * a.ldp + r;
+    *pm = valid ? exp2f((*pm - lse) * LOG2E_F) * scale : 0.f;
   }
 }
 

@@ -226,7 +226,8 @@ struct Plan {
   int64_t chunk, n_chunks;
   int64_t tile_w;  // partial tile width (columns)
   int64_t ntile, lde, ldp;
-  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, off_xpart, total;
+  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, off_xpart, off_lse, total;
+  bool keep;  // FLCE_FLAG_KEEP_LOGITS / FLCE_FLAG_FROM_KEPT: one chunk, lse kept in the workspace
   bool facc;
   int64_t xpart_elems;  // grad_X split-K partials (fp32 elements)
 };
@@ -246,6 +247,12 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
   const int64_t per_row = p->lde * esz + p->ntile * 8 + 4;
   int64_t chunk = opt && opt->chunk_rows > 0 ? round_up(opt->chunk_rows, 128) : 0;
   const int64_t bt_r = std::max<int64_t>(round_up(std::max<int64_t>(BT, 1), 128), 128);
+  p->keep = opt && (opt->flags & (FLCE_FLAG_KEEP_LOGITS | FLCE_FLAG_FROM_KEPT));
+  if (p->keep) {
+    // the whole batch is one chunk whose store outlives the call
+    if (bt_r > kMaxChunk) return FLCE_ERR_INVALID_ARG;
+    chunk = bt_r;
+  }
   if (chunk == 0) {
     if (opt && opt->workspace_limit_bytes > 0) {
       chunk = (opt->workspace_limit_bytes / per_row) / 128 * 128;
@@ -277,6 +284,7 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
   p->off_facc = o; o = align256(o + (p->facc ? (size_t)V * H * 4 : 0));
   p->xpart_elems = dtype == FLCE_BF16 ? gradx_partial_elems(BT, H, V, chunk) : 0;
   p->off_xpart = o; o = align256(o + (size_t)p->xpart_elems * 4);
+  p->off_lse = o; o = align256(o + (p->keep ? (size_t)chunk * 4 : 0));
   p->total = o;
   return FLCE_OK;
 }
@@ -488,6 +496,12 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     if (grad_X && BT > 0 && (!is_aligned(grad_X->data, 16) || grad_X->stride[0] % 8)) return FLCE_ERR_INVALID_ARG;
     if (grad_W && (!is_aligned(grad_W->data, 16) || grad_W->stride[0] % 8)) return FLCE_ERR_INVALID_ARG;
   }
+  // two-phase use: a forward pass that keeps its chunk store, then gradients from it
+  const bool keep = opt && (opt->flags & FLCE_FLAG_KEEP_LOGITS);
+  const bool from_kept = opt && (opt->flags & FLCE_FLAG_FROM_KEPT);
+  if (keep && from_kept) return FLCE_ERR_INVALID_ARG;
+  if ((keep || from_kept) && !opt->workspace) return FLCE_ERR_INVALID_ARG;  // must outlive the call
+  if (keep && (grad_X || grad_W || sharded)) return FLCE_ERR_INVALID_ARG;
   const bool want_gx = grad_X != nullptr && BT > 0;
   const bool want_gw = grad_W != nullptr || sharded;
   const bool need_rowloss = reduction != FLCE_NONE && !(opt && opt->row_loss);
@@ -536,6 +550,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   float* facc = pl.facc ? reinterpret_cast<float*>(base + pl.off_facc) : nullptr;
   float* xpart = pl.xpart_elems ? reinterpret_cast<float*>(base + pl.off_xpart) : nullptr;
   float* lse_out = opt ? opt->lse : nullptr;
+  float* lse_kept = pl.keep ? reinterpret_cast<float*>(base + pl.off_lse) : nullptr;
   const int64_t* tgt = static_cast<const int64_t*>(target->data);
 
   // A0: N (always run: it also flags targets outside [0, V))
@@ -550,7 +565,14 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     const int64_t r0 = c * pl.chunk;
     const int rows = (int)std::min<int64_t>(pl.chunk, BT - r0);
     const int64_t* tgt_c = tgt + r0;
-    if (dt == FLCE_BF16) {
+    if (from_kept) {
+      // the store and tile maxima are those the KEEP_LOGITS call left; turn the
+      // maxima into factors with this call's row_grad and scale
+      FactorArgs a{tgt_c, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, lse_kept, nvalid, reduction,
+                   row_grad ? row_grad + r0 : nullptr};
+      st = L.run(2, [&] { factor_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
+      if (st != FLCE_OK) return st;
+    } else if (dt == FLCE_BF16) {
       const __nv_bfloat16* Xc = static_cast<const __nv_bfloat16*>(X->data) + r0 * ldx;
       const __nv_bfloat16* Wp = static_cast<const __nv_bfloat16*>(W->data);
       __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
@@ -588,12 +610,15 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       if (st != FLCE_OK) return st;
     }
     // A3
-    {
+    if (!from_kept) {
       CombineArgs a{tgt_c, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, ps, zt,
-                    row_loss + r0, lse_out ? lse_out + r0 : nullptr, nvalid, reduction,
-                    row_grad ? row_grad + r0 : nullptr};
+                    row_loss + r0, keep ? lse_kept : (lse_out ? lse_out + r0 : nullptr), nvalid, reduction,
+                    row_grad ? row_grad + r0 : nullptr, keep ? 1 : 0};
       st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
       if (st != FLCE_OK) return st;
+      if (keep && lse_out &&
+          cudaMemcpyAsync(lse_out, lse_kept, (size_t)rows * 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+        return FLCE_ERR_CUDA;
     }
     if (!want_gx && !want_gw) continue;
     // A4
@@ -744,7 +769,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       }
     }
   }
-  if (reduction != FLCE_NONE) {
+  if (reduction != FLCE_NONE && !from_kept) {
     st = L.run(5, [&] {
       finalize_loss_kernel<<<1, 1024, 0, stream>>>(row_loss, BT, nvalid, reduction,
                                                    static_cast<float*>(loss->data));

@@ -24,11 +24,16 @@ responses and rows B..2B-1 the rejected ones of the same prompts. Prompt and
 padding positions carry ignore_index. KTO takes [N, T] sequences and a 0/1
 `desirable` vector instead of pairs.
 
-Every loss depends on the logits only through the per-token losses l_t, so it
-runs as two passes of the CUDA path: a forward pass that returns l_t
-(reduction 'none', no gradients), O(batch) tensor work that gives the loss and
-g_t = dLoss/dl_t, and a second pass with row_grad = g_t that produces grad_X
-and grad_W. The logits are never materialised in either pass.
+Every loss depends on the logits only through the per-token losses l_t. The
+CUDA path gives l_t (reduction 'none'), O(batch) tensor work gives the loss and
+g_t = dLoss/dl_t, and the gradients are those of sum_t g_t * l_t (row_grad).
+Two schedules:
+  single pass (default while the batch's chunk store fits keep_limit_bytes):
+    forward_keep keeps the bf16 store of the whole batch, and backward_from_kept
+    takes the gradients from it: 6*BT*H*V tensor FLOPs;
+  two passes: a forward pass, then the chunked fused path again with row_grad:
+    8*BT*H*V tensor FLOPs, with the chunked path's memory.
+The fp32 logits are never materialised in either.
 """
 from __future__ import annotations
 
@@ -36,7 +41,7 @@ from typing import Optional
 
 import torch
 
-from .api import fused_linear_cross_entropy
+from .api import backward_from_kept, forward_keep, fused_linear_cross_entropy, keep_workspace_bytes
 
 KINDS = ("dpo", "orpo", "cpo", "simpo", "kto")
 
@@ -83,19 +88,30 @@ def preference_loss_from_logps(kind: str, lp: torch.Tensor, count: torch.Tensor,
 def fused_linear_preference_loss(kind: str, weight: torch.Tensor, x: torch.Tensor, target: torch.Tensor,
                                  ignore_index: int = -100, beta: float = 0.1, gamma: float = 0.5, lam: float = 0.1,
                                  ref_logps: Optional[torch.Tensor] = None, desirable: Optional[torch.Tensor] = None,
-                                 want_grad_X: bool = True, want_grad_W: bool = True, **kw):
+                                 want_grad_X: bool = True, want_grad_W: bool = True, single_pass="auto",
+                                 keep_limit_bytes: int = 2 << 30, **kw):
     """(loss, grad_x, grad_weight) of a preference loss over lm_head logits x weight^T.
 
     x [N, T, H] or [N*T, H] with target [N, T]; N = 2B (pairs) or the KTO
     sequence count. Returns grads shaped like x and weight.
+    single_pass: True, False, or "auto" (when the batch's store fits
+    keep_limit_bytes and the batch is at most 32768 tokens).
     """
     if kind not in KINDS:
         raise ValueError(f"kind must be one of {KINDS}")
     n_seq = target.shape[0]
     X = x.reshape(-1, x.shape[-1])
     t = target.reshape(-1)
-    row_loss, _, _ = fused_linear_cross_entropy(X, weight, t, ignore_index=ignore_index, reduction="none",
-                                                want_grad_X=False, want_grad_W=False, **kw)
+    if single_pass == "auto":
+        single_pass = (not kw and X.shape[0] <= 32768 and
+                       keep_workspace_bytes(X.shape[0], X.shape[1], weight.shape[0],
+                                            "bf16" if X.dtype == torch.bfloat16 else "f32") <= keep_limit_bytes)
+    kept = None
+    if single_pass:
+        row_loss, kept = forward_keep(X, weight, t, ignore_index=ignore_index, reduction="none")
+    else:
+        row_loss, _, _ = fused_linear_cross_entropy(X, weight, t, ignore_index=ignore_index, reduction="none",
+                                                    want_grad_X=False, want_grad_W=False, **kw)
     # O(batch) sequence-level part: loss and its gradient w.r.t. each token's loss
     # (grad mode is forced on: autograd.Function.forward runs with it off)
     with torch.enable_grad():
@@ -108,9 +124,13 @@ def fused_linear_preference_loss(kind: str, weight: torch.Tensor, x: torch.Tenso
                                           ref_logps=None if ref_logps is None else ref_logps.double(),
                                           desirable=desirable)
         (g,) = torch.autograd.grad(loss, rl)
-    _, gX, gW = fused_linear_cross_entropy(X, weight, t, ignore_index=ignore_index, reduction="none",
-                                           row_grad=g.float(), want_grad_X=want_grad_X, want_grad_W=want_grad_W,
-                                           **kw)
+    if kept is not None:
+        gX, gW = backward_from_kept(kept, reduction="none", row_grad=g.float(), want_grad_X=want_grad_X,
+                                    want_grad_W=want_grad_W)
+    else:
+        _, gX, gW = fused_linear_cross_entropy(X, weight, t, ignore_index=ignore_index, reduction="none",
+                                               row_grad=g.float(), want_grad_X=want_grad_X,
+                                               want_grad_W=want_grad_W, **kw)
     return loss.detach().float(), (gX.reshape(x.shape) if gX is not None else None), gW
 
 

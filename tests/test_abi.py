@@ -194,3 +194,35 @@ def test_grad_W_shard_options_are_validated(lib):
         rc = lib.flce_fwd_bwd_ex(ctypes.byref(X), ctypes.byref(W), ctypes.byref(tg), -100, 0, ctypes.byref(loss),
                                  None, None, None, ctypes.byref(o), ctypes.byref(st))
         assert rc == 1, (rows, n, ld)
+
+
+def test_keep_flags_are_validated(lib):
+    X = _t(FAKE, B.BF16, (64, 128))
+    W = _t(FAKE, B.BF16, (1000, 128))
+    tg = _t(FAKE, B.I64, (64,))
+    loss = _t(FAKE, B.F32, ())
+    gW = _t(FAKE, B.BF16, (1000, 128))
+
+    def call(flags, workspace, grad_W=None, X=X, tg=tg):
+        o = B.FlceOptions()
+        lib.flce_options_init(ctypes.byref(o))
+        o.flags = flags
+        if workspace:
+            o.workspace, o.workspace_bytes = FAKE * 256, 1 << 40
+        return lib.flce_fwd_bwd_ex(ctypes.byref(X), ctypes.byref(W), ctypes.byref(tg), -100, 0,
+                                   ctypes.byref(loss), None, ctypes.byref(grad_W) if grad_W else None, None,
+                                   ctypes.byref(o), None)
+
+    assert call(B.FLAG_KEEP_LOGITS, False) == 1                      # the store needs a caller workspace
+    assert call(B.FLAG_FROM_KEPT, False) == 1
+    assert call(B.FLAG_KEEP_LOGITS | B.FLAG_FROM_KEPT, True) == 1    # one phase at a time
+    assert call(B.FLAG_KEEP_LOGITS, True, grad_W=gW) == 1            # the forward phase takes no gradients
+    big_X, big_t = _t(FAKE, B.BF16, (40000, 128)), _t(FAKE, B.I64, (40000,))
+    assert call(B.FLAG_KEEP_LOGITS, True, X=big_X, tg=big_t) == 1    # more rows than one chunk holds
+    st = B.FlceStats()
+    o = B.FlceOptions()
+    lib.flce_options_init(ctypes.byref(o))
+    o.flags = B.FLAG_KEEP_LOGITS
+    assert lib.flce_plan(4096, 4096, 128256, B.BF16, 1, ctypes.byref(o), ctypes.byref(st)) == 0
+    assert st.n_chunks == 1 and st.chunk_rows == 4096
+    assert st.workspace_bytes >= 4096 * 128256 * 2

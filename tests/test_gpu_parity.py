@@ -381,3 +381,50 @@ def test_cross_entropy_one_pass_matches_multipass(monkeypatch):
     assert rel_err(l1.item(), l2.item()) <= 1e-5
     d = (g1.float() - g2.float()).abs().max().item()
     assert d <= 2 ** -8 * g2.float().abs().max().item(), d
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("reduction", ["mean", "none"])
+def test_keep_then_gradients_from_kept(dtype, reduction):
+    """forward_keep + backward_from_kept (the logits GEMM once) against the oracle
+    and against the one-call path with the same row_grad."""
+    w = WORKLOADS["tiny"] if dtype == "f32" else WORKLOADS["llama3_8b_seq"]
+    d = make_inputs(w, BT=700, H=256, V=3000)
+    X, W, t = to_dev(d)
+    g = np.random.default_rng(2).standard_normal(700).astype(np.float32)
+    rg = torch.from_numpy(g).cuda() if reduction == "none" else None
+    lse = torch.empty(700, dtype=torch.float32, device="cuda")
+    loss, kept = L().forward_keep(X, W, t, reduction=reduction, lse=lse)
+    gX, gW = L().backward_from_kept(kept, reduction=reduction, row_grad=rg)
+    torch.cuda.synchronize()
+    ref = oracle.flce(d["X"], d["W"], d["target"], reduction=reduction, row_grad=g if rg is not None else None)
+    tol = TOL[dtype]
+    if reduction == "none":
+        np.testing.assert_allclose(loss.cpu().numpy(), ref["loss"], rtol=tol["loss"], atol=tol["loss"])
+    else:
+        assert rel_err(loss.item(), ref["loss"]) <= tol["loss"]
+    assert_grad_close(gX, ref["grad_X"], dtype, "grad_X (kept)")
+    assert_grad_close(gW, ref["grad_W"], dtype, "grad_W (kept)")
+    z = d["X"].astype(np.float64) @ d["W"].astype(np.float64).T
+    ref_lse = np.log(np.exp(z - z.max(1, keepdims=True)).sum(1)) + z.max(1)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=1e-4, atol=1e-3)
+    # the one-call path with the same reduction and row_grad: same dz, same grad_X rows
+    l2, gX2, gW2 = L().fused_linear_cross_entropy(X, W, t, reduction=reduction, row_grad=rg, chunk_rows=768)
+    torch.cuda.synchronize()
+    assert torch.equal(gX, gX2)
+    assert torch.allclose(loss, l2, rtol=1e-6, atol=0)
+    with pytest.raises(RuntimeError, match="already used"):
+        L().backward_from_kept(kept)
+
+
+def test_module_none_keep_logits():
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
+    X, W, t = to_dev(d)
+    X = X.reshape(2, 128, 128).clone().requires_grad_(True)
+    W = W.clone().requires_grad_(True)
+    rows = L().FusedLinearCrossEntropyLoss(reduction="none", keep_logits=True)(W, X, t.reshape(2, 128))
+    g = torch.randn(2, 128, device="cuda", generator=torch.Generator(device="cuda").manual_seed(1))
+    rows.backward(g)
+    ref = oracle.flce(d["X"], d["W"], d["target"], reduction="none", row_grad=g.reshape(-1).cpu().numpy())
+    assert_grad_close(X.grad.reshape(256, 128), ref["grad_X"], "bf16", "module keep grad_X")
+    assert_grad_close(W.grad, ref["grad_W"], "bf16", "module keep grad_W")

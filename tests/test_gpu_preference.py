@@ -28,8 +28,9 @@ def _case(B=4, T=48, H=256, V=3000):
     return d["X"], d["W"], t
 
 
+@pytest.mark.parametrize("single_pass", [True, False])
 @pytest.mark.parametrize("kind", KINDS)
-def test_preference_loss_parity(kind):
+def test_preference_loss_parity(kind, single_pass):
     from linear_cross_entropy_04_b200.preference import fused_linear_preference_loss
 
     X, W, t = _case()
@@ -45,7 +46,7 @@ def test_preference_loss_parity(kind):
     Xd = torch.from_numpy(X).to(torch.bfloat16).cuda().reshape(N, T, -1)
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     loss, gX, gW = fused_linear_preference_loss(kind, Wd, Xd, torch.from_numpy(t).cuda(), beta=0.1, gamma=0.5,
-                                                lam=0.1, **dkw)
+                                                lam=0.1, single_pass=single_pass, **dkw)
     torch.cuda.synchronize()
     assert rel_err(loss.item(), ref["loss"]) <= 1e-3, (loss.item(), ref["loss"])
     assert_grad_close(gX.reshape(N * T, -1), ref["grad_X"], "bf16", f"{kind} grad_X")
@@ -65,3 +66,22 @@ def test_preference_module_matches_function():
     assert rel_err(loss.item(), ref["loss"]) <= 1e-3
     assert_grad_close(Xd.grad.reshape(N * T, -1), ref["grad_X"], "bf16", "orpo module grad_X")
     assert_grad_close(Wd.grad, ref["grad_W"], "bf16", "orpo module grad_W")
+
+
+def test_single_pass_matches_two_pass():
+    """The kept-store schedule and the recompute schedule give the same loss and
+    gradients up to the order of grad_W's chunk additions."""
+    from linear_cross_entropy_04_b200.preference import fused_linear_preference_loss
+
+    X, W, t = _case(B=8, T=64, H=256, V=5000)  # 1024 tokens: two chunks in the recompute schedule
+    N, T = t.shape
+    Xd = torch.from_numpy(X).to(torch.bfloat16).cuda().reshape(N, T, -1)
+    Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
+    td = torch.from_numpy(t).cuda()
+    l1, x1, w1 = fused_linear_preference_loss("simpo", Wd, Xd, td, single_pass=True)
+    l2, x2, w2 = fused_linear_preference_loss("simpo", Wd, Xd, td, single_pass=False, chunk_rows=512)
+    torch.cuda.synchronize()
+    assert l1.item() == l2.item()
+    assert torch.equal(x1, x2)  # grad_X rows do not depend on the chunking
+    d = (w1.float() - w2.float()).abs().max().item()
+    assert d <= 2 ** -7 * w2.float().abs().max().item(), d
