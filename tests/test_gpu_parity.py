@@ -428,3 +428,25 @@ def test_module_none_keep_logits():
     ref = oracle.flce(d["X"], d["W"], d["target"], reduction="none", row_grad=g.reshape(-1).cpu().numpy())
     assert_grad_close(X.grad.reshape(256, 128), ref["grad_X"], "bf16", "module keep grad_X")
     assert_grad_close(W.grad, ref["grad_W"], "bf16", "module keep grad_W")
+
+
+@pytest.mark.parametrize("V,BT", [(50000, 1000), (128256, 400), (152064, 300)])
+@pytest.mark.parametrize("want_lse", [False, True])
+def test_cross_entropy_many_rows_in_place(V, BT, want_lse):
+    """Hundreds of rows (many clusters per SM over the launch), ignored rows
+    interleaved and in runs, in place, with and without the lse output."""
+    z, t = _ce_inputs(V % 89, BT, V, ignore_every=3)
+    t[5:9] = IGNORE_INDEX
+    td = torch.from_numpy(t).cuda()
+    zd = z.cuda()
+    lse = torch.empty(BT, dtype=torch.float32, device="cuda") if want_lse else None
+    loss, g = L().cross_entropy(zd, td, inplace=True, lse=lse)
+    torch.cuda.synchronize()
+    z64 = z.double().numpy()
+    ref = oracle.cross_entropy(z64, t)
+    assert rel_err(loss.item(), ref["loss"]) <= TOL["bf16"]["loss"]
+    assert_grad_close(g, ref["dz"], "bf16", "dz (many rows)")
+    assert g.data_ptr() == zd.data_ptr()
+    if want_lse:
+        ref_lse = np.log(np.exp(z64 - z64.max(1, keepdims=True)).sum(1)) + z64.max(1)
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=1e-5, atol=1e-4)
