@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_seq")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-slots", type=int, default=2, help="device buffer sets of the host pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--chunk-rows", type=int, default=0)
@@ -597,7 +598,7 @@ def main():
         torch.cuda.empty_cache()
         houts = [(torch.empty((), dtype=torch.float32).pin_memory(), torch.empty_like(Xh).pin_memory(),
                   torch.empty_like(Wh).pin_memory()) for _ in range(2)]
-        pipe = HostPipeline(w.BT, w.H, w.V, dtype=dt, **kw)
+        pipe = HostPipeline(w.BT, w.H, w.V, dtype=dt, slots=args.e2e_slots, **kw)
         for i in range(2):
             pipe.submit(Xh, Wh, th, houts[i % 2])
         pipe.synchronize()
@@ -610,10 +611,32 @@ def main():
         h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size() + th.numel() * 8
         d2h = 4 + houts[0][1].numel() * houts[0][1].element_size() + houts[0][2].numel() * houts[0][2].element_size()
         e2e = {"value": w.BT * args.e2e_steps / wall, "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * wall / args.e2e_steps,
+               "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * wall / args.e2e_steps, "slots": args.e2e_slots,
                "how": "public API (HostPipeline): pinned host X, W, target copied in and loss, grad_X, grad_W "
                       "copied back every step; copies overlap compute across steps (wall clock)"}
-        del pipe, Xh, Wh, th, houts
+        del pipe
+        # the copies' own bound: one step's uploads and downloads issued together on
+        # two streams (PCIe carries both directions at once), no compute
+        up = [torch.empty_like(Xh, device=dev), torch.empty_like(Wh, device=dev), torch.empty_like(th, device=dev)]
+        dn = [torch.empty_like(houts[0][1], device=dev), torch.empty_like(houts[0][2], device=dev)]
+        s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        best = float("inf")
+        for _ in range(4):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            with torch.cuda.stream(s1):
+                for d_, h_ in zip(up, (Xh, Wh, th)):
+                    d_.copy_(h_, non_blocking=True)
+            with torch.cuda.stream(s2):
+                houts[0][1].copy_(dn[0], non_blocking=True)
+                houts[0][2].copy_(dn[1], non_blocking=True)
+            torch.cuda.synchronize()
+            best = min(best, time.perf_counter() - t0)
+        e2e["pcie_bound"] = {"value": w.BT / best, "unit": UNIT, "ms_per_step": 1e3 * best,
+                             "frac": e2e["value"] / (w.BT / best),
+                             "how": "one step's host-to-device and device-to-host copies issued together "
+                                    "on two streams, best of 4 (wall clock)"}
+        del up, dn, Xh, Wh, th, houts
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
