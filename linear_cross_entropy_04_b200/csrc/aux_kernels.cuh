@@ -375,7 +375,10 @@ __global__ void __launch_bounds__(256) ce_grad_kernel(CeGradArgs<T> a) {
 // 64 registers per thread let 4 CTAs share an SM; exponentials use the PTX
 // ex2.approx.ftz instruction (results below 2^-126 flush to 0).
 constexpr int CER_THREADS = 256;
-constexpr int CER_VPT = 8;                              // 8-element vectors per thread
+#ifndef FLCE_CER_VPT
+#define FLCE_CER_VPT 8
+#endif
+constexpr int CER_VPT = FLCE_CER_VPT;                   // 8-element vectors per thread
 constexpr int CER_SLICE = CER_THREADS * CER_VPT * 8;    // max columns per CTA
 constexpr int CER_MAX_CLUSTER = 16;
 #ifndef FLCE_CER_MIN_BLOCKS
