@@ -36,22 +36,34 @@ def _lib_flce(X, W, target, ignore_index, reduction, n_valid, want_grad_X, want_
                                       n_valid=n_valid, want_grad_X=want_grad_X, want_grad_W=want_grad_W, **kw)
 
 
-class _PeerShards:
-    """This rank's grad_W shard in symmetric memory and every rank's shard mapped here.
+def shard_rows_for(V: int, world: int) -> int:
+    """Rows of grad_W each rank owns: V / world rounded up to a multiple of 32,
+    so that no 32-row output box of the grad_W GEMM straddles two owners."""
+    return ((-(-V // world)) + 31) // 32 * 32
 
-    shard_rows = V / world rounded up to a multiple of 32, so that no 32-row
-    output box of the grad_W GEMM straddles two owners."""
+
+def owned_rows(V: int, shard_rows: int, rank: int) -> int:
+    """How many of rank's shard_rows are real grad_W rows (the last owners may hold fewer, or none)."""
+    return max(0, min(shard_rows, V - rank * shard_rows))
+
+
+class _PeerShards:
+    """This rank's grad_W shard in symmetric memory and every rank's shard mapped
+    here (buf, peers, shard_rows, rank, barrier(): the interface the fused path uses)."""
 
     def __init__(self, V, H, dtype, device, group):
         import torch.distributed._symmetric_memory as symm_mem
 
         world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
-        self.shard_rows = ((-(-V // world)) + 31) // 32 * 32
+        self.shard_rows = shard_rows_for(V, world)
         self.buf = symm_mem.empty(self.shard_rows, H, dtype=dtype, device=device)
         self.hdl = symm_mem.rendezvous(self.buf, group if group is not None else dist.group.WORLD)
         self.peers = [self.hdl.get_buffer(r, (self.shard_rows, H), dtype) for r in range(world)]
         self.V = V
+
+    def barrier(self):
+        self.hdl.barrier()  # device-side, on the current stream
 
 
 _shards_cache = {}
@@ -68,7 +80,7 @@ def dp_fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torc
                                   ignore_index: int = -100, reduction: str = "mean",
                                   group: Optional[dist.ProcessGroup] = None,
                                   want_grad_X: bool = True, want_grad_W: bool = True,
-                                  shard_grad_W: bool = False, fused_grad_W: bool = False,
+                                  shard_grad_W: bool = False, fused_grad_W: bool = False, shards=None,
                                   count_fn: Callable = _lib_count, flce_fn: Callable = _lib_flce, **kw):
     """Global loss, this rank's grad_X, and grad_W summed over ranks.
 
@@ -79,11 +91,14 @@ def dp_fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torc
     grad_W GEMM: each output tile is added, over NVLink, into the shard of the
     rank that owns its rows (torch symmetric memory), and this rank gets its
     shard, rows [r*S, (r+1)*S) with S = V/world rounded up to 32. The shards
-    are zeroed before and read after a barrier across ranks.
+    are zeroed before and read after a barrier across ranks. `shards` may
+    supply them (buf, peers, shard_rows, rank, barrier()); by default they are
+    symmetric-memory buffers.
     Every rank takes the same collective steps in the same order.
     """
     if fused_grad_W:
-        return _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, **kw)
+        return _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, shards, count_fn,
+                                flce_fn, **kw)
     n_valid = None
     if reduction == "mean":
         n_valid = count_fn(target, W.shape[0], ignore_index).to(torch.int64).reshape(())
@@ -111,21 +126,17 @@ def dp_fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torc
     return loss, gX, gW
 
 
-def _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, **kw):
-    from .api import count_valid, fused_linear_cross_entropy
-
+def _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, shards, count_fn, flce_fn, **kw):
     V, H = W.shape
-    sh = _peer_shards(V, H, W.dtype, W.device, group)
+    sh = shards if shards is not None else _peer_shards(V, H, W.dtype, W.device, group)
     n_valid = None
     if reduction == "mean":
-        n_valid = count_valid(target, V, ignore_index).reshape(())
+        n_valid = count_fn(target, V, ignore_index).to(torch.int64).reshape(())
         dist.all_reduce(n_valid, group=group)
     sh.buf.zero_()
-    sh.hdl.barrier()  # every rank's shard is zero before any rank adds into it
-    loss, gX, _ = fused_linear_cross_entropy(X, W, target, ignore_index=ignore_index, reduction=reduction,
-                                             n_valid=n_valid, want_grad_X=want_grad_X,
-                                             grad_w_shards=sh.peers, shard_rows=sh.shard_rows, **kw)
-    sh.hdl.barrier()  # every rank's additions into this rank's shard have landed
+    sh.barrier()  # every rank's shard is zero before any rank adds into it
+    loss, gX, _ = flce_fn(X, W, target, ignore_index, reduction, n_valid, want_grad_X, False,
+                          grad_w_shards=sh.peers, shard_rows=sh.shard_rows, **kw)
+    sh.barrier()  # every rank's additions into this rank's shard have landed
     dist.all_reduce(loss, group=group)
-    rows = max(0, min(sh.shard_rows, V - sh.rank * sh.shard_rows))
-    return loss, gX, sh.buf[:rows]
+    return loss, gX, sh.buf[:owned_rows(V, sh.shard_rows, sh.rank)]

@@ -25,7 +25,7 @@ def _free_port():
 
 def _case(case):
     rng = np.random.default_rng(7)
-    BT, H, V = 37, 6, 20
+    BT, H, V = 37, 6, (70 if case == "wide" else 20)
     X = rng.standard_normal((BT, H))
     W = rng.standard_normal((V, H)) * 0.5
     t = rng.integers(0, V, BT)
@@ -150,3 +150,122 @@ def test_a_dead_rank_makes_the_next_collective_fail_instead_of_hanging():
         if p.is_alive():
             p.kill()
     assert msg.startswith("error"), msg
+
+
+# ---- fused grad_W reduce-scatter: the host logic (shard sizes, zeroing, the two
+# barriers, the slice each rank keeps), with CPU shards in shared memory standing
+# in for symmetric memory and the oracle standing in for the device call, whose
+# per-box adds into the owner shards are emulated under a lock (in L2 they are
+# atomic element-wise adds).
+
+def test_shard_sizes():
+    from linear_cross_entropy_04_b200.dp import owned_rows, shard_rows_for
+
+    assert shard_rows_for(128256, 8) == 16032 and shard_rows_for(70, 2) == 64 and shard_rows_for(20, 2) == 32
+    for V, world in ((128256, 8), (152064, 3), (70, 2), (20, 2), (33, 4)):
+        S = shard_rows_for(V, world)
+        assert S % 32 == 0 and S * world >= V
+        assert sum(owned_rows(V, S, r) for r in range(world)) == V
+
+
+class _CpuShards:
+    """Shards in shared memory. The emulated device call adds into them from a
+    background thread (device work is asynchronous); barrier() first waits for
+    this rank's pending adds, as a device-side barrier orders after the work
+    already on its stream, then meets the other ranks."""
+
+    def __init__(self, bufs, rank, shard_rows):
+        self.buf, self.peers, self.shard_rows, self.rank = bufs[rank], bufs, shard_rows, rank
+        self.pending = []
+
+    def barrier(self):
+        import torch.distributed as dist
+
+        for th in self.pending:
+            th.join()
+        self.pending.clear()
+        dist.barrier()
+
+
+def _fused_worker(rank, world, port, reduction, bufs, lock, q):
+    import sys
+    import time
+
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import oracle
+    from linear_cross_entropy_04_b200.dp import dp_fused_linear_cross_entropy, owned_rows
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        X, W, t, split = _case("wide")
+        V = W.shape[0]
+        sl = slice(0, split) if rank == 0 else slice(split, None)
+        count_fn, _ = _oracle_fns()
+
+        shards = _CpuShards(bufs, rank, bufs[0].shape[0])
+
+        def flce_fn(Xr, Wr, tr, ii, red, nv, want_gx, want_gw, grad_w_shards=None, shard_rows=0):
+            import threading
+
+            r = oracle.flce(Xr.numpy(), Wr.numpy(), tr.numpy(), ignore_index=ii, reduction=red,
+                            n_valid=None if nv is None else int(nv))
+
+            def adds():
+                if rank == 1:
+                    time.sleep(0.5)  # a slow rank: its adds land late
+                with lock:
+                    for k, shard in enumerate(grad_w_shards):
+                        n = owned_rows(V, shard_rows, k)
+                        shard[:n] += torch.from_numpy(r["grad_W"][k * shard_rows:k * shard_rows + n])
+
+            th = threading.Thread(target=adds)
+            th.start()
+            shards.pending.append(th)
+            return torch.tensor(r["loss"], dtype=torch.float64), torch.from_numpy(r["grad_X"]), None
+
+        if rank == 1:
+            time.sleep(0.5)  # late to zero its shard: rank 0 must not add into it before
+        loss, gX, gW = dp_fused_linear_cross_entropy(
+            torch.from_numpy(X[sl]), torch.from_numpy(W), torch.from_numpy(t[sl]), reduction=reduction,
+            fused_grad_W=True, shards=shards, count_fn=count_fn, flce_fn=flce_fn)
+        res = (rank, float(loss), gX.numpy(), gW.clone().numpy())
+        for th in shards.pending:
+            th.join()
+        q.put(res)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("reduction", ["mean", "sum"])
+def test_dp_fused_grad_W_reduce_scatter_host_logic(reduction):
+    import oracle
+    from linear_cross_entropy_04_b200.dp import shard_rows_for
+
+    X, W, t, split = _case("wide")
+    V, H = W.shape
+    S = shard_rows_for(V, 2)
+    ctx = mp.get_context("spawn")
+    bufs = [torch.full((S, H), float("nan"), dtype=torch.float64).share_memory_() for _ in range(2)]
+    lock = ctx.Lock()
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_fused_worker, args=(r, 2, port, reduction, bufs, lock, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    out = {}
+    for _ in range(2):
+        r, loss, gX, gW = q.get(timeout=120)
+        out[r] = (loss, gX, gW)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ref = oracle.flce(X, W, t, reduction=reduction)
+    assert out[0][2].shape == (S, H) and out[1][2].shape == (V - S, H)
+    for r in range(2):
+        assert abs(out[r][0] - ref["loss"]) < 1e-12 * max(1.0, abs(ref["loss"]))
+    np.testing.assert_allclose(np.concatenate([out[0][2], out[1][2]]), ref["grad_W"], atol=1e-14)
+    np.testing.assert_allclose(np.concatenate([out[0][1], out[1][1]]), ref["grad_X"], atol=1e-15)
