@@ -108,8 +108,9 @@ typedef enum {
 typedef struct {
   int64_t chunk_rows;            /* rows per chunk; 0 = chosen from workspace_limit_bytes.
                                     Rounded up to a multiple of 128. */
-  int64_t workspace_limit_bytes; /* chunk store budget; 0 = at most 512 MiB and at most half
-                                    the rows, so two or more chunks whenever BT > 128 */
+  int64_t workspace_limit_bytes; /* chunk store budget; 0 = at most 512 MiB but at least 2048
+                                    rows, and at most half the rows, so two or more chunks
+                                    whenever BT > 128 */
   void* workspace;               /* optional caller-owned device workspace (256-byte aligned) */
   int64_t workspace_bytes;       /* its size in bytes */
   int32_t grad_w_accum;          /* flce_gradw_accum */

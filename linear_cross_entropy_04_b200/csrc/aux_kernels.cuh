@@ -57,8 +57,12 @@ __global__ void count_valid_kernel(const int64_t* __restrict__ target, int64_t B
 }
 
 // ------------------------------------------------------------------ A3
-// Block = 256 threads = 8 warps over 32 rows: lane <-> row, warp w merges
-// tiles w, w+8, ... so every partial load is a coalesced 128-byte read.
+// Block = CB_THREADS threads = CB_WARPS warps over 32 rows: lane <-> row, warp
+// w merges tiles w, w + CB_WARPS, ... so every partial load is a coalesced
+// 128-byte read, and 32 warps per 32 rows keep enough loads in flight for a
+// long row of tiles (a grid of only rows / 32 blocks).
+constexpr int CB_WARPS = 32;
+constexpr int CB_THREADS = CB_WARPS * 32;
 struct CombineArgs {
   const int64_t* target;  // chunk row 0
   int64_t ignore_index, V;
@@ -76,14 +80,14 @@ struct CombineArgs {
   int skip_factors;       // 1: leave the tile maxima in part_m (factor_kernel turns them later)
 };
 
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
-  __shared__ float sm_m[8][32], sm_s[8][32], sm_lse[32];
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(CombineArgs a) {
+  __shared__ float sm_m[CB_WARPS][32], sm_s[CB_WARPS][32], sm_lse[32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int r = blockIdx.x * 32 + lane;
   const bool row_ok = r < a.rows;
   float M = -INFINITY, S = 0.f;
   if (row_ok) {
-    for (int j = w; j < a.ntile; j += 8) {
+    for (int j = w; j < a.ntile; j += CB_WARPS) {
       const float m = a.part_m[(int64_t)j * a.ldp + r];
       const float s = a.part_s[(int64_t)j * a.ldp + r];
       if (m > M) {
@@ -99,9 +103,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   __syncthreads();
   if (w == 0) {
     float Mt = -INFINITY;
-    for (int k = 0; k < 8; ++k) Mt = fmaxf(Mt, sm_m[k][lane]);
+    for (int k = 0; k < CB_WARPS; ++k) Mt = fmaxf(Mt, sm_m[k][lane]);
     float St = 0.f;
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < CB_WARPS; ++k)
       if (sm_m[k][lane] != -INFINITY) St += sm_s[k][lane] * exp2f((sm_m[k][lane] - Mt) * LOG2E_F);
     const float lse = Mt + logf(St);
     sm_lse[lane] = lse;
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     const bool valid = target_valid(a.target[r], a.V, a.ignore_index);
     const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
     const float lse = sm_lse[lane];
-    for (int j = w; j < a.ntile; j += 8) {
+    for (int j = w; j < a.ntile; j += CB_WARPS) {
       float* pm = a.part_m + (int64_t)j * a.ldp + r;
       *pm = valid ? exp2f((*pm - lse) * LOG2E_F) * scale : 0.f;
     }
@@ -138,14 +142,14 @@ struct FactorArgs {
   const float* row_grad;  // optional [rows]
 };
 
-__global__ void __launch_bounds__(256) factor_kernel(FactorArgs a) {
+__global__ void __launch_bounds__(CB_THREADS) factor_kernel(FactorArgs a) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int r = blockIdx.x * 32 + lane;
   if (r >= a.rows) return;
   const bool valid = target_valid(a.target[r], a.V, a.ignore_index);
   const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
   const float lse = a.lse[r];
-  for (int j = w; j < a.ntile; j += 8) {
+  for (int j = w; j < a.ntile; j += CB_WARPS) {
     float* pm = a.part_m + (int64_t)j * a.ldp + r;
     *pm = valid ? exp2f((*pm - lse) * LOG2E_F) * scale : 0.f;
   }

@@ -35,6 +35,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kDefaultLimit = 512ll << 20;
 constexpr int64_t kMaxChunk = 32768;
+constexpr int64_t kMinDefaultChunk = 2048;
 
 struct DeviceCtx {
   bool init = false;
@@ -257,10 +258,12 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
     if (opt && opt->workspace_limit_bytes > 0) {
       chunk = (opt->workspace_limit_bytes / per_row) / 128 * 128;
     } else {
-      // default: at most 512 MiB of chunk store, and at most half of the rows,
-      // so the logits of the whole batch are never held at once
-      chunk = std::min<int64_t>((kDefaultLimit / per_row) / 128 * 128,
-                                round_up(ceil_div(std::max<int64_t>(BT, 1), 2), 128));
+      // default: at most 512 MiB of chunk store, but at least 2048 rows (grad_W's
+      // K: shorter chunks leave its tiles epilogue-bound and repeat the per-chunk
+      // passes), and at most half of the rows, so the logits of the whole batch
+      // are never held at once
+      const int64_t half = round_up(ceil_div(std::max<int64_t>(BT, 1), 2), 128);
+      chunk = std::min<int64_t>(std::max<int64_t>((kDefaultLimit / per_row) / 128 * 128, kMinDefaultChunk), half);
     }
     if (chunk < 128) chunk = 128;
     if (chunk > kMaxChunk) chunk = kMaxChunk;
@@ -570,7 +573,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       // maxima into factors with this call's row_grad and scale
       FactorArgs a{tgt_c, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, lse_kept, nvalid, reduction,
                    row_grad ? row_grad + r0 : nullptr};
-      st = L.run(2, [&] { factor_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
+      st = L.run(2, [&] { factor_kernel<<<(unsigned)ceil_div(rows, 32), CB_THREADS, 0, stream>>>(a); });
       if (st != FLCE_OK) return st;
     } else if (dt == FLCE_BF16) {
       const __nv_bfloat16* Xc = static_cast<const __nv_bfloat16*>(X->data) + r0 * ldx;
@@ -614,7 +617,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       CombineArgs a{tgt_c, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, ps, zt,
                     row_loss + r0, keep ? lse_kept : (lse_out ? lse_out + r0 : nullptr), nvalid, reduction,
                     row_grad ? row_grad + r0 : nullptr, keep ? 1 : 0};
-      st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
+      st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), CB_THREADS, 0, stream>>>(a); });
       if (st != FLCE_OK) return st;
       if (keep && lse_out &&
           cudaMemcpyAsync(lse_out, lse_kept, (size_t)rows * 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
@@ -891,7 +894,7 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
     const int rows = (int)std::min<int64_t>(65535 * 32, BT - r0);
     CombineArgs a{tgt + r0, ignore_index, V, rows, (int)ntile, ldp, pm + r0, ps + r0, zt + r0, rl + r0, lse + r0, nv, reduction,
                   row_grad ? row_grad + r0 : nullptr};
-    st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a); });
+    st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), CB_THREADS, 0, stream>>>(a); });
     if (st != FLCE_OK) return st;
   }
   if (grad) {
@@ -1031,7 +1034,7 @@ flce_status run_ce_noalloc(const flce_tensor* Z, const flce_tensor* target, int6
   for (int64_t r0 = 0; r0 < BT; r0 += 65535 * 32) {
     const int rows = (int)std::min<int64_t>(65535 * 32, BT - r0);
     CombineArgs a{tgt + r0, ignore_index, V, rows, (int)ntile, ldp, pm + r0, ps + r0, zt + r0, rl + r0, lse + r0, nv, reduction};
-    combine_kernel<<<(unsigned)ceil_div(rows, 32), 256, 0, stream>>>(a);
+    combine_kernel<<<(unsigned)ceil_div(rows, 32), CB_THREADS, 0, stream>>>(a);
   }
   if (grad) {
     for (int64_t r0 = 0; r0 < BT; r0 += 65535) {
