@@ -201,6 +201,12 @@ FLCE_API flce_status flce_count_valid(const flce_tensor* target, int64_t V, int6
  *   logits tensor itself (in-place gradient replacement).
  * opt may be NULL; only opt->n_valid, opt->row_loss, opt->lse and opt->row_grad are read.
  * FLCE_NONE as for flce_fwd_bwd (loss is f32 [BT]).
+ * bf16 logits with V up to 16 * 16384 (8 * 16384 on a device that cannot hold
+ * a 16-CTA cluster) take one pass: a thread-block cluster per row reads the
+ * logits once and writes the gradient once, with a workspace of N and the
+ * per-row losses only. f32 logits and longer rows take three passes (per-tile
+ * partials, row combine, gradient) with a per-(row, 1024-column tile) partials
+ * workspace. The workspace comes from the library's memory pool.
  */
 FLCE_API flce_status flce_cross_entropy(const flce_tensor* logits, const flce_tensor* target,
                                int64_t ignore_index, int32_t reduction, flce_tensor* loss,
@@ -257,9 +263,11 @@ FLCE_API flce_status flce_get_device_error(flce_stream_t stream, uint32_t* err);
  * recorded events and writes, for each phase p < n_phases, the summed
  * milliseconds to ms[p] and the number of timed launches to count[p] (either
  * may be NULL). reset != 0 clears the record afterwards. Phases:
- *   0 count valid rows, 1 logits GEMM + online-softmax epilogue,
- *   2 row combine + loss, 3 in-place dlogits, 4 grad_X / grad_W GEMMs,
- *   5 final loss reduction.
+ *   0 count valid rows, 1 logits GEMM + online-softmax epilogue (for
+ *   flce_cross_entropy: the per-tile partials, or the one-pass row kernel),
+ *   2 row combine + loss (or the factors of a FLCE_FLAG_FROM_KEPT call),
+ *   3 in-place dlogits (flce_cross_entropy: the gradient pass),
+ *   4 grad_X / grad_W GEMMs, 5 final loss reduction.
  */
 #define FLCE_NUM_PHASES 6
 FLCE_API flce_status flce_phase_times(double* ms, int32_t* count, int32_t n_phases, int32_t reset);
