@@ -450,3 +450,24 @@ def test_cross_entropy_many_rows_in_place(V, BT, want_lse):
     if want_lse:
         ref_lse = np.log(np.exp(z64 - z64.max(1, keepdims=True)).sum(1)) + z64.max(1)
         np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=1e-5, atol=1e-4)
+
+
+# The engine's alternative paths, each forced by its switch: the single-CTA
+# engine, grad_X and grad_W in one launch or two, and grad_X split over K
+# (few output tiles, a long K: 2 x 2 tiles over K = 9000 / 64 blocks).
+@pytest.mark.parametrize("env", [{"FLCE_ENGINE": "1sm"}, {"FLCE_GRAD_LAUNCH": "combined"},
+                                 {"FLCE_GRAD_LAUNCH": "split"}, {"FLCE_GRADX_SPLITK": "1"},
+                                 {"FLCE_ENGINE": "1sm", "FLCE_GRAD_LAUNCH": "combined"}],
+                         ids=["1sm", "combined", "split", "splitk", "1sm-combined"])
+def test_engine_variants_match_oracle(monkeypatch, env):
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=500, H=512, V=9000)
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=384)
+    torch.cuda.synchronize()
+    assert L().device_error() == 0
+    ref = oracle.flce(d["X"], d["W"], d["target"])
+    assert rel_err(loss.item(), ref["loss"]) <= TOL["bf16"]["loss"]
+    assert_grad_close(gX, ref["grad_X"], "bf16", f"grad_X {env}")
+    assert_grad_close(gW, ref["grad_W"], "bf16", f"grad_W {env}")
