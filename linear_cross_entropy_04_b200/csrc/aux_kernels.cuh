@@ -7,8 +7,13 @@
 //   dlogits_kernel       in place over the chunk store: e * factor - onehot*scale,
 //                        0 for ignored rows (A4, "in-place gradient replacement"
 //                        of the paper review's 主な発見)
+//   factor_kernel        combine's factor step alone, for gradients taken from
+//                        a kept forward pass (FLCE_FLAG_FROM_KEPT)
 //   finalize_loss_kernel fixed-order sum of the per-row losses, times 1/N or 1
-//   ce_partials_kernel   logits given: per-(row, tile) partials read from z
+//   ce_row_cluster_kernel logits given, bf16: one cluster of CTAs per row, z
+//                        read once and dz written once
+//   ce_partials_kernel   logits given (f32, or rows too long for a cluster):
+//                        per-(row, tile) partials read from z
 //   ce_grad_kernel       logits given: dz from z and lse, optionally in place
 //   simt_gemm_kernel     fp32 FMA GEMM with the same epilogues as the tcgen05
 //                        engine, for fp32 inputs where TF32 tensor cores would

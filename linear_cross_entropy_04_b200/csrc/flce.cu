@@ -7,9 +7,11 @@
 //   A1+A2  logits GEMM z = X_c W^T with the online-softmax epilogue
 //   A3     row combine: lse, per-row loss, per-tile factors
 //   A4     in-place dlogits over the chunk store (技術原理 > 原地操作)
-//   A5+A6  grad_X_c = dz W and grad_W (+)= dz^T X_c in one persistent launch
+//   A5+A6  grad_X_c = dz W and grad_W (+)= dz^T X_c, in one persistent launch
+//          or two (grad_combined)
 // then one fixed-order loss reduction. The full BT x V logits never exist:
-// the store holds one chunk of rows at a time.
+// the store holds one chunk of rows at a time (except on request: the
+// two-phase flags keep the whole batch as one chunk between two calls).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
