@@ -14,6 +14,12 @@ the non-ignored row count before the loss, then of the loss and of grad_W.
 
 --impl reference times the float64 CPU oracle on bounded samples of the same
 workload (rank 0 only); it is the slow baseline the pages' method is exact to.
+
+Other paths (one GPU, their own JSON lines):
+  --path ce                 logits-given cross-entropy vs torch cross_entropy + backward
+  --path preference --kind  a fused-linear preference-loss step vs PyTorch on materialised logits
+--dp-fused-grad-w (N > 1) replaces the grad_W all-reduce by the reduce-scatter the
+grad_W GEMM does itself into symmetric-memory shards.
 """
 from __future__ import annotations
 

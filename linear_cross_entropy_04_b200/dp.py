@@ -11,9 +11,11 @@ exchanges, done with the process group's collectives (NCCL over NVLink on GPUs):
                         ranks is the global mean;
   3. all_reduce(grad_W) (or reduce_scatter of its rows, for sharded grad_W).
 
-grad_X stays local. The per-rank compute is the CUDA library; `count_fn` and
-`flce_fn` exist so that host-side tests can run the exchange logic on CPU
-ranks with a stand-in compute.
+grad_X stays local. With fused_grad_W the third exchange disappears: the
+grad_W GEMM adds each output box into the owner rank's shard itself (NVLink,
+torch symmetric memory). The per-rank compute is the CUDA library; `count_fn`,
+`flce_fn` and `shards` exist so that host-side tests can run the exchange
+logic on CPU ranks with a stand-in compute.
 """
 from __future__ import annotations
 
