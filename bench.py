@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama3_8b_seq")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=24,
+                    help="host-buffer steps timed end to end (the pipeline's fill and drain are included)")
     ap.add_argument("--e2e-slots", type=int, default=2, help="device buffer sets of the host pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -619,7 +620,8 @@ def main():
         e2e = {"value": w.BT * args.e2e_steps / wall, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * wall / args.e2e_steps, "slots": args.e2e_slots,
                "how": "public API (HostPipeline): pinned host X, W, target copied in and loss, grad_X, grad_W "
-                      "copied back every step; copies overlap compute across steps (wall clock)"}
+                      "copied back every step; copies overlap compute across steps (wall clock, the "
+                      "pipeline's fill and drain included)"}
         del pipe
         # the copies' own bound: one step's uploads and downloads issued together on
         # two streams (PCIe carries both directions at once), no compute
