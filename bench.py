@@ -247,14 +247,14 @@ def calibrate_rows(d, Wf, target_s, cap):
     t40 = oracle_sample(d, 40, Wf)
     per_row = max((t40 - t8) / 32, 1e-6)
     fixed = max(t8 - 8 * per_row, 0.0)
-    return int(max(8, min(cap, (target_s - fixed) / per_row)))
+    return int(min(cap, max(8, (target_s - fixed) / per_row)))
 
 
 def cpu_baseline(d, target_s):
     import numpy as np
 
     Wf = d["W"].astype(np.float64)
-    rows = calibrate_rows(d, Wf, target_s, 4096)
+    rows = calibrate_rows(d, Wf, target_s, min(4096, d["BT"]))
     t = oracle_sample(d, rows, Wf)
     return {"value": rows / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"first {rows} tokens of the workload, full fwd+bwd per token in float64 NumPy "
@@ -273,7 +273,7 @@ def run_reference(args):
     w = WORKLOADS[args.workload]
     d = make_inputs(w)
     Wf = d["W"].astype(np.float64)
-    rows = calibrate_rows(d, Wf, 150.0 / max(1, args.steps + args.warmup), 4096)
+    rows = calibrate_rows(d, Wf, 150.0 / max(1, args.steps + args.warmup), min(4096, d["BT"]))
     for _ in range(args.warmup):
         oracle_sample(d, rows, Wf)
     tot = 0.0

@@ -51,3 +51,20 @@ def test_oracle_sample_sizing_separates_fixed_cost(bench, monkeypatch):
     assert bench.calibrate_rows(None, None, 12.0, 4096) == 2200
     assert bench.calibrate_rows(None, None, 100.0, 4096) == 4096
     assert bench.calibrate_rows(None, None, 0.5, 4096) == 8
+
+
+def test_reference_arm_runs_on_the_host_and_samples_at_most_the_batch():
+    """bench.py --impl reference: the oracle as it stands, one JSON line, a
+    sample no larger than the workload's batch."""
+    import json
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["dtype"] == "f64" and line["config"]["workload"] == "tiny"
+    assert line["config"]["sample_tokens_per_step"] <= 512
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["value"] > 0 and line["unit"] == "tokens/s"
