@@ -1,0 +1,72 @@
+"""The fused data-parallel grad_W path on one rank: its symmetric-memory calls
+(buffer, rendezvous, peer view, device barrier) run for real on one GPU.
+
+With one rank the owner of every grad_W row is this rank, so the shard it
+keeps must equal the plain path's grad_W bit for bit (the first chunk's adds
+into the zeroed shard are exact, as the plain path's first store is), and the
+loss and grad_X must be identical. Runs in a spawned child so the process
+group does not outlive the test.
+"""
+import datetime
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _child(port, q):
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from linear_cross_entropy_04_b200 import fused_linear_cross_entropy
+    from linear_cross_entropy_04_b200.dp import dp_fused_linear_cross_entropy
+    from linear_cross_entropy_04_b200.inputs import WORKLOADS, make_inputs
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=700, H=256, V=3000)
+        X = torch.from_numpy(d["X"]).to(torch.bfloat16).cuda()
+        W = torch.from_numpy(d["W"]).to(torch.bfloat16).cuda()
+        t = torch.from_numpy(d["target"]).cuda()
+        l1, x1, w1 = fused_linear_cross_entropy(X, W, t, chunk_rows=256)
+        l2, x2, w2 = dp_fused_linear_cross_entropy(X, W, t, fused_grad_W=True, chunk_rows=256)
+        torch.cuda.synchronize()
+        q.put(("ok", float(l1), float(l2), bool(torch.equal(x1, x2)), tuple(w2.shape), bool(torch.equal(w1, w2))))
+    except Exception as e:  # noqa: BLE001 - report, do not hang the parent
+        q.put(("error", f"{type(e).__name__}: {e}"))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_fused_grad_W_path_on_one_rank():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_child, args=(_free_port(), q))
+    p.start()
+    res = q.get(timeout=300)
+    p.join(timeout=60)
+    assert res[0] == "ok", res
+    _, l1, l2, same_x, shape, same_w = res
+    assert l1 == l2 and same_x
+    assert shape == (3000, 256) and same_w
+    assert p.exitcode == 0
