@@ -1,5 +1,6 @@
-"""The fused data-parallel grad_W path on one rank: its symmetric-memory calls
-(buffer, rendezvous, peer view, device barrier) run for real on one GPU.
+"""The data-parallel paths on one rank, for real on one GPU: the fused grad_W
+path's symmetric-memory calls (buffer, rendezvous, peer view, device barrier)
+and the collective path's NCCL all-reduces and reduce-scatter.
 
 With one rank the owner of every grad_W row is this rank, so the shard it
 keeps must equal the plain path's grad_W bit for bit (the first chunk's adds
@@ -48,15 +49,24 @@ def _child(port, q):
         t = torch.from_numpy(d["target"]).cuda()
         l1, x1, w1 = fused_linear_cross_entropy(X, W, t, chunk_rows=256)
         l2, x2, w2 = dp_fused_linear_cross_entropy(X, W, t, fused_grad_W=True, chunk_rows=256)
+        # the collective path (NCCL all-reduces, and the reduce-scatter of sharded grad_W)
+        l3, x3, w3 = dp_fused_linear_cross_entropy(X, W, t, chunk_rows=256)
+        l4, x4, w4 = dp_fused_linear_cross_entropy(X, W, t, shard_grad_W=True, chunk_rows=256)
+        ls, _, ws = fused_linear_cross_entropy(X, W, t, reduction="sum", chunk_rows=256)
+        l5, _, w5 = dp_fused_linear_cross_entropy(X, W, t, reduction="sum", chunk_rows=256)
         torch.cuda.synchronize()
-        q.put(("ok", float(l1), float(l2), bool(torch.equal(x1, x2)), tuple(w2.shape), bool(torch.equal(w1, w2))))
+        collective = (float(l3) == float(l1) and torch.equal(x3, x1) and torch.equal(w3, w1) and
+                      float(l4) == float(l1) and torch.equal(w4, w1) and
+                      float(l5) == float(ls) and torch.equal(w5, ws))
+        q.put(("ok", float(l1), float(l2), bool(torch.equal(x1, x2)), tuple(w2.shape), bool(torch.equal(w1, w2)),
+               bool(collective)))
     except Exception as e:  # noqa: BLE001 - report, do not hang the parent
         q.put(("error", f"{type(e).__name__}: {e}"))
     finally:
         dist.destroy_process_group()
 
 
-def test_fused_grad_W_path_on_one_rank():
+def test_data_parallel_paths_on_one_rank():
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     ctx = mp.get_context("spawn")
@@ -66,7 +76,8 @@ def test_fused_grad_W_path_on_one_rank():
     res = q.get(timeout=300)
     p.join(timeout=60)
     assert res[0] == "ok", res
-    _, l1, l2, same_x, shape, same_w = res
+    _, l1, l2, same_x, shape, same_w, collective = res
     assert l1 == l2 and same_x
     assert shape == (3000, 256) and same_w
+    assert collective  # all-reduce and reduce-scatter paths equal the single-process call
     assert p.exitcode == 0
