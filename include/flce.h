@@ -30,6 +30,11 @@
  *    ignore_index) set a bit of the device error word, read with
  *    flce_get_device_error(); such rows are treated as ignored. Nothing traps.
  *  - No C++ exception crosses this interface.
+ *  - Calls may come from several host threads at once: the library's own
+ *    state (the per-device context and the phase-timing record) is guarded by
+ *    a mutex, and each call takes its own workspace. A caller-provided
+ *    workspace (flce_options.workspace) must not be shared by calls that may
+ *    run on the GPU at the same time.
  */
 #ifndef FLCE_H
 #define FLCE_H
