@@ -34,6 +34,16 @@ int main(void) {
   if (flce_fwd_bwd(&X, &W, &t, -100, FLCE_MEAN, &loss, NULL, NULL, NULL) != FLCE_ERR_UNSUPPORTED_DTYPE)
     return fail("dtype mix");
   if (strcmp(flce_status_string(FLCE_OK), "ok") != 0) return fail("status string");
+  /* two-phase planning: one chunk holding the whole batch, in a caller workspace */
+  flce_options keep;
+  flce_options_init(&keep);
+  keep.flags = FLCE_FLAG_KEEP_LOGITS;
+  flce_stats kst;
+  if (flce_plan(4096, 4096, 128256, FLCE_BF16, 1, &keep, &kst) != FLCE_OK) return fail("keep plan");
+  if (kst.n_chunks != 1 || kst.chunk_rows != 4096) return fail("keep chunking");
+  if (kst.workspace_bytes < kst.materialized_logits_bytes) return fail("keep workspace holds the store");
+  if (flce_plan(40000, 4096, 128256, FLCE_BF16, 1, &keep, &kst) != FLCE_ERR_INVALID_ARG)
+    return fail("keep limit");
   printf("ok\n");
   return 0;
 }
