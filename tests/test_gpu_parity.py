@@ -471,3 +471,32 @@ def test_engine_variants_match_oracle(monkeypatch, env):
     assert rel_err(loss.item(), ref["loss"]) <= TOL["bf16"]["loss"]
     assert_grad_close(gX, ref["grad_X"], "bf16", f"grad_X {env}")
     assert_grad_close(gW, ref["grad_W"], "bf16", f"grad_W {env}")
+
+
+# Degenerate shapes of the method: a one-class vocabulary (every row's loss and
+# gradient are exactly 0), two classes (the logistic loss), a single row, and
+# the smallest hidden size with an odd vocabulary.
+@pytest.mark.parametrize("wl,BT,H,V", [("llama3_8b_seq", 1, 64, 100), ("llama3_8b_seq", 40, 64, 2),
+                                       ("llama3_8b_seq", 5, 8, 7), ("tiny", 1, 16, 2), ("tiny", 9, 8, 3)])
+def test_degenerate_shapes(wl, BT, H, V):
+    run_case(make_inputs(WORKLOADS[wl], BT=BT, H=H, V=V))
+
+
+@pytest.mark.parametrize("wl", ["llama3_8b_seq", "tiny"])
+def test_one_class_vocabulary_is_exactly_zero(wl):
+    d = make_inputs(WORKLOADS[wl], BT=40, H=64, V=1)
+    d["target"][d["target"] != IGNORE_INDEX] = 0
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t)
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0
+    assert torch.all(gX == 0) and torch.all(gW == 0)
+    # logits given: rows padded to 16 bytes, as the ABI requires; the one-pass
+    # kernel's exp2(z*log2e - max*log2e) leaves the rounding of z*log2e, so the
+    # result is 0 to fp32 precision rather than exactly
+    buf = torch.zeros(7, 8, dtype=X.dtype)
+    buf[:, 0] = torch.randn(7).to(X.dtype)
+    z = buf.cuda()[:, :1]
+    lz, dz = L().cross_entropy(z, torch.zeros(7, dtype=torch.int64, device="cuda"))
+    torch.cuda.synchronize()
+    assert abs(lz.item()) <= 1e-6 and dz.float().abs().max().item() <= 1e-6
