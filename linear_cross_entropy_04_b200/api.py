@@ -103,6 +103,8 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                  ctypes.byref(tgW) if tgW is not None else None,
                                  B.stream_handle(stream), ctypes.byref(o), ctypes.byref(st))
     B.check(rc, "flce_fwd_bwd_ex")
+    if ws is not None and stream is not None:
+        ws.record_stream(stream)  # allocated on the current stream, used on `stream`
     if host:
         if host_out is not None:
             hl, hx, hw = host_out
@@ -160,6 +162,8 @@ def forward_keep(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor, ignore_
     B.check(B.lib().flce_fwd_bwd_ex(ctypes.byref(tX), ctypes.byref(tW), ctypes.byref(tt), int(ignore_index),
                                     _RED[reduction], ctypes.byref(tl), None, None, B.stream_handle(stream),
                                     ctypes.byref(o), None), "flce_fwd_bwd_ex (keep)")
+    if stream is not None:
+        ws.record_stream(stream)  # allocated on the current stream, used on `stream`
     return loss, KeptLogits(X, W, target, ignore_index, ws, n_valid)
 
 
@@ -185,6 +189,9 @@ def backward_from_kept(kept: KeptLogits, reduction: str = "mean", row_grad: Opti
                                     ctypes.byref(tgX) if tgX is not None else None,
                                     ctypes.byref(tgW) if tgW is not None else None,
                                     B.stream_handle(stream), ctypes.byref(o), None), "flce_fwd_bwd_ex (from kept)")
+    # the workspace was allocated on the forward's stream; keep the allocator
+    # from reusing it before this call's kernels, possibly on another stream, finish
+    kept.workspace.record_stream(stream if stream is not None else torch.cuda.current_stream(X.device))
     kept.workspace = None
     return gX, gW
 
