@@ -190,6 +190,14 @@ FLCE_API flce_status flce_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, 
                       const flce_options* opt, flce_stats* out);
 
 /*
+ * Host-only: the workspace bytes flce_fwd_bwd_ex would use for this shape and
+ * options with grad_W requested (flce_plan's workspace_bytes), i.e. the size a
+ * caller-provided opt->workspace needs. 0 for an empty batch; (size_t)-1 if
+ * the arguments are invalid. Touches no GPU.
+ */
+FLCE_API size_t flce_workspace_bytes(int64_t BT, int64_t H, int64_t V, int32_t dtype, const flce_options* opt);
+
+/*
  * N, the count of rows whose target is not ignore_index, written as int64
  * to the DEVICE pointer n_valid_out on `stream`. Targets outside [0,V) that
  * are not ignore_index set FLCE_DEVERR_TARGET_RANGE and are not counted.

@@ -72,6 +72,8 @@ _SIGS = {
                                        ctypes.c_void_p, _P(FlceOptions), _P(FlceStats)]),
     "flce_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
                                  ctypes.c_int32, _P(FlceOptions), _P(FlceStats)]),
+    "flce_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                               _P(FlceOptions)]),
     "flce_count_valid": (ctypes.c_int, [_P(FlceTensor), ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                         ctypes.c_void_p]),
     "flce_cross_entropy": (ctypes.c_int, [_P(FlceTensor), _P(FlceTensor), ctypes.c_int64, ctypes.c_int32,

@@ -1104,6 +1104,12 @@ flce_status flce_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, int32_t w
   return FLCE_OK;
 }
 
+size_t flce_workspace_bytes(int64_t BT, int64_t H, int64_t V, int32_t dtype, const flce_options* opt) {
+  flce_stats st;
+  if (flce_plan(BT, H, V, dtype, 1, opt, &st) != FLCE_OK) return (size_t)-1;
+  return (size_t)st.workspace_bytes;
+}
+
 flce_status flce_count_valid(const flce_tensor* target, int64_t V, int64_t ignore_index,
                              int64_t* n_valid_out, flce_stream_t stream) {
   if (!target || !n_valid_out || V <= 0) return FLCE_ERR_INVALID_ARG;

@@ -34,6 +34,8 @@ int main(void) {
   if (flce_fwd_bwd(&X, &W, &t, -100, FLCE_MEAN, &loss, NULL, NULL, NULL) != FLCE_ERR_UNSUPPORTED_DTYPE)
     return fail("dtype mix");
   if (strcmp(flce_status_string(FLCE_OK), "ok") != 0) return fail("status string");
+  if (flce_workspace_bytes(4096, 4096, 128256, FLCE_BF16, &opt) != (size_t)st.workspace_bytes)
+    return fail("workspace bytes");
   /* two-phase planning: one chunk holding the whole batch, in a caller workspace */
   flce_options keep;
   flce_options_init(&keep);

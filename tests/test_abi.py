@@ -229,3 +229,21 @@ def test_keep_flags_are_validated(lib):
     assert lib.flce_plan(4096, 4096, 128256, B.BF16, 1, ctypes.byref(o), ctypes.byref(st)) == 0
     assert st.n_chunks == 1 and st.chunk_rows == 4096
     assert st.workspace_bytes >= 4096 * 128256 * 2
+
+
+def test_workspace_bytes_matches_the_plan(lib):
+    """flce_workspace_bytes is flce_plan's workspace figure with grad_W requested."""
+    for BT, H, V, dt in ((4096, 4096, 128256, B.BF16), (512, 256, 4096, B.F32), (16384, 2048, 256000, B.BF16)):
+        st = B.FlceStats()
+        assert lib.flce_plan(BT, H, V, dt, 1, None, ctypes.byref(st)) == 0
+        assert lib.flce_workspace_bytes(BT, H, V, dt, None) == st.workspace_bytes > 0
+    o = B.FlceOptions()
+    lib.flce_options_init(ctypes.byref(o))
+    o.grad_w_accum = B.GRADW_ACCUM_FP32
+    st = B.FlceStats()
+    assert lib.flce_plan(4096, 4096, 128256, B.BF16, 1, ctypes.byref(o), ctypes.byref(st)) == 0
+    assert lib.flce_workspace_bytes(4096, 4096, 128256, B.BF16, ctypes.byref(o)) == st.workspace_bytes
+    assert lib.flce_workspace_bytes(0, 4096, 128256, B.BF16, None) == 0          # empty batch
+    invalid = ctypes.c_size_t(-1).value
+    assert lib.flce_workspace_bytes(10, 0, 10, B.BF16, None) == invalid          # H = 0
+    assert lib.flce_workspace_bytes(10, 8, 10, B.I64, None) == invalid           # not a float dtype
