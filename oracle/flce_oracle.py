@@ -22,7 +22,7 @@ approximation. So the result the fused method must reach is the plain one:
 The call shape follows the low-level API of "Liger-Kernel 項目詳細介紹"
 (使用方法 > 3. 低級 API 方式): loss_fn(weight [V,H], input [BT,H], target [BT]).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * mean divides by N, the count of non-ignored rows;
   * 'none' returns the per-row losses (0 for ignored rows), as the torch loss
     modules the pages' low-level API mirrors do; with an upstream gradient
