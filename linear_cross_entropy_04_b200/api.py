@@ -18,12 +18,19 @@ _RED = {"mean": B.MEAN, "sum": B.SUM, "none": B.NONE}
 _ACC = {"output": B.GRADW_ACCUM_OUTPUT, "fp32": B.GRADW_ACCUM_FP32}
 
 
+def _check_reduction(reduction):
+    if reduction not in _RED:
+        raise ValueError(f"reduction must be one of {sorted(_RED)}, not {reduction!r}")
+
+
 def _options(chunk_rows=0, workspace_limit_bytes=0, grad_w_accum="output", flags=0,
              n_valid=None, row_loss=None, lse=None, workspace=None, row_grad=None):
     o = B.FlceOptions()
     B.lib().flce_options_init(ctypes.byref(o))
     o.chunk_rows = int(chunk_rows)
     o.workspace_limit_bytes = int(workspace_limit_bytes)
+    if grad_w_accum not in _ACC:
+        raise ValueError(f"grad_w_accum must be one of {sorted(_ACC)}, not {grad_w_accum!r}")
     o.grad_w_accum = _ACC[grad_w_accum]
     o.flags = int(flags)
     o.n_valid = None if n_valid is None else n_valid.data_ptr()
@@ -63,6 +70,7 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     The library's workspace is taken from torch's caching allocator.
     Returns (loss [scalar fp32], grad_X or None, grad_W or None[, stats]).
     """
+    _check_reduction(reduction)
     host = not X.is_cuda
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -150,6 +158,7 @@ def forward_keep(X: torch.Tensor, W: torch.Tensor, target: torch.Tensor, ignore_
                  lse: Optional[torch.Tensor] = None, stream=None):
     """Loss of cross-entropy over X W^T with the batch's chunk store kept for
     backward_from_kept (FLCE_FLAG_KEEP_LOGITS). Returns (loss, KeptLogits)."""
+    _check_reduction(reduction)
     loss = torch.empty((X.shape[0],) if reduction == "none" else (), dtype=torch.float32, device=X.device)
     o = _options(flags=B.FLAG_KEEP_LOGITS, n_valid=n_valid, lse=lse)
     st = B.FlceStats()
@@ -172,6 +181,7 @@ def backward_from_kept(kept: KeptLogits, reduction: str = "mean", row_grad: Opti
     """grad_X, grad_W from a forward_keep (FLCE_FLAG_FROM_KEPT): the gradients
     of sum_i row_grad_i * l_i * (1/N or 1) without running the logits GEMM again.
     The kept workspace is released afterwards."""
+    _check_reduction(reduction)
     X, W, t = kept.X, kept.W, kept.target
     if kept.workspace is None:
         raise RuntimeError("the kept logits were already used")
@@ -201,6 +211,7 @@ def cross_entropy(logits: torch.Tensor, target: torch.Tensor, ignore_index: int 
                   n_valid: Optional[torch.Tensor] = None, row_loss: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, row_grad: Optional[torch.Tensor] = None, stream=None):
     """Cross-entropy of given logits [BT, V]; the gradient may replace the logits in place."""
+    _check_reduction(reduction)
     loss = torch.empty((logits.shape[0],) if reduction == "none" else (), dtype=torch.float32,
                        device=logits.device)
     grad = None

@@ -247,3 +247,20 @@ def test_workspace_bytes_matches_the_plan(lib):
     invalid = ctypes.c_size_t(-1).value
     assert lib.flce_workspace_bytes(10, 0, 10, B.BF16, None) == invalid          # H = 0
     assert lib.flce_workspace_bytes(10, 8, 10, B.I64, None) == invalid           # not a float dtype
+
+
+def test_python_api_rejects_bad_option_strings():
+    """Bad option strings fail in Python with a clear error, before any device work."""
+    import torch
+
+    from linear_cross_entropy_04_b200 import api
+
+    X, W, t = torch.zeros(4, 8), torch.zeros(10, 8), torch.zeros(4, dtype=torch.int64)
+    with pytest.raises(ValueError, match="reduction"):
+        api.fused_linear_cross_entropy(X, W, t, reduction="avg")
+    with pytest.raises(ValueError, match="reduction"):
+        api.cross_entropy(torch.zeros(4, 10), t, reduction="total")
+    with pytest.raises(ValueError, match="reduction"):
+        api.forward_keep(X, W, t, reduction="mean_")
+    with pytest.raises(ValueError, match="grad_w_accum"):
+        api.plan(4, 8, 10, grad_w_accum="fp16")
