@@ -522,3 +522,60 @@ def test_preference_against_torch_float64(kind):
     assert abs(r["loss"] - L.item()) < 1e-12
     np.testing.assert_allclose(r["grad_X"], Xt.grad.numpy(), rtol=1e-9, atol=1e-14)
     np.testing.assert_allclose(r["grad_W"], Wt.grad.numpy(), rtol=1e-9, atol=1e-14)
+
+
+# ------------------------------------------------ preference-oracle mutations
+
+def _pref_pins():
+    def finite_differences():
+        for k in PREF:
+            test_preference_finite_differences(k)
+
+    def closed_forms():
+        test_preference_closed_forms_for_identical_pairs()
+
+    def torch_float64():
+        for k in PREF:
+            test_preference_against_torch_float64(k)
+
+    return [finite_differences, closed_forms, torch_float64]
+
+
+def _pref_mutants():
+    """Plausible mistakes in the preference oracle, each planted in one helper."""
+    real_seq = po.sequence_logps
+    real_ltg = po.loss_and_token_grad
+
+    def logps_unmasked(row_loss, target, n_seq, ignore_index=-100):
+        _, _, valid = real_seq(row_loss, target, n_seq, ignore_index)
+        ones = np.ones_like(valid)
+        return -np.asarray(row_loss, dtype=np.float64).reshape(n_seq, -1).sum(1), ones.sum(1), ones
+
+    def logsig_sign(u):
+        return -np.logaddexp(0.0, u)
+
+    def sigmoid_flipped(u):
+        return 1.0 / (1.0 + np.exp(u))
+
+    def token_grad_sign(*a, **k):
+        loss, g = real_ltg(*a, **k)
+        return loss, -g
+
+    def token_grad_halved(*a, **k):
+        loss, g = real_ltg(*a, **k)
+        return loss, 0.5 * g
+
+    return [("sequence_logps", logps_unmasked), ("_logsig", logsig_sign), ("_sigmoid", sigmoid_flipped),
+            ("loss_and_token_grad", token_grad_sign), ("loss_and_token_grad", token_grad_halved)]
+
+
+@pytest.mark.parametrize("name,fn", _pref_mutants(), ids=lambda x: x if isinstance(x, str) else x.__name__)
+def test_preference_mutants_are_caught(monkeypatch, name, fn):
+    monkeypatch.setattr(po, name, fn)
+    caught = []
+    for pin in _pref_pins():
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"no preference pin caught the planted mistake in {name} ({fn.__name__})"
