@@ -63,7 +63,25 @@ def parse():
     ap.add_argument("--kind", default="dpo", choices=["dpo", "orpo", "cpo", "simpo", "kto"],
                     help="preference loss for --path preference")
     ap.add_argument("--seq-len", type=int, default=512, help="tokens per sequence for --path preference")
+    ap.add_argument("--BT", type=int, default=0, help="profiling: cut the workload to this many tokens")
+    ap.add_argument("--H", type=int, default=0, help="profiling: hidden size override")
+    ap.add_argument("--V", type=int, default=0, help="profiling: vocabulary size override")
     return ap.parse_args()
+
+
+def workload(args):
+    """The named workload, or the same recipe at the --BT/--H/--V sizes (small
+    cases for profiling); an overridden workload is renamed after its sizes."""
+    import dataclasses
+
+    from linear_cross_entropy_04_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    over = {k: getattr(args, k) for k in ("BT", "H", "V") if getattr(args, k)}
+    if not over:
+        return w
+    w = dataclasses.replace(w, **over)
+    return dataclasses.replace(w, name=f"{args.workload} recipe at {w.BT}x{w.H}x{w.V}")
 
 
 def load_peaks():
@@ -179,7 +197,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- recorded ncu traffic
 
-KERNEL_SOURCES = ["linear_cross_entropy_04_b200/csrc/" + f for f in ("tc_gemm2.cuh", "tc_gemm.cuh", "ptx.cuh")]
+# everything that decides what the captured launches do: the kernels, and the
+# host code that picks their chunking, tile order and launch split
+KERNEL_SOURCES = ["linear_cross_entropy_04_b200/csrc/" + f
+                  for f in ("tc_gemm2.cuh", "tc_gemm.cuh", "ptx.cuh", "aux_kernels.cuh", "flce.cu")]
 
 
 def kernel_source_hash():
@@ -276,7 +297,7 @@ def run_reference(args):
 
     from linear_cross_entropy_04_b200.inputs import WORKLOADS, make_inputs
 
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     d = make_inputs(w)
     Wf = d["W"].astype(np.float64)
     rows = calibrate_rows(d, Wf, 150.0 / max(1, args.steps + args.warmup), min(4096, d["BT"]))
@@ -313,7 +334,7 @@ def run_ce(args):
 
     import numpy as np
 
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(0)
     z0 = (torch.randn(w.BT, w.V, device=dev, generator=g) * 1.28).to(torch.bfloat16)
@@ -395,7 +416,7 @@ def run_preference(args):
     from linear_cross_entropy_04_b200.inputs import IGNORE_INDEX, WORKLOADS, make_inputs
     from linear_cross_entropy_04_b200.preference import fused_linear_preference_loss, preference_loss_from_logps
 
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     T = args.seq_len
     n_seq = w.BT // T
     assert n_seq >= 2 and n_seq % 2 == 0, "BT / seq_len must be an even number of sequences"
@@ -470,10 +491,12 @@ def run_preference(args):
             "memory_ratio_torch_over_ours": res["torch"]["peak_extra_bytes"] / max(res["ours"]["peak_extra_bytes"], 1),
             "loss_rel_diff_vs_torch": rel, "ours": res["ours"], "torch": res["torch"],
             "roofline": {"bound": "tensor", "achieved": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12,
-                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops"],
                          "traffic": None, "algorithmic_flops": useful,
-                         "frac_of_burst_peak": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                         "peak_kind": f"{peaks['source']} burst bf16",
+                         "frac_of_sustained_peak": useful / (res["ours"]["ms_per_step"] / 1e3) / 1e12
+                         / peaks["bf16_tflops_sustained"],
                          "note": "useful 6*BT*H*V; the single-pass schedule executes exactly these, the "
                                  "two-pass one (batches whose store exceeds the keep budget) 8*BT*H*V"},
             "clocks": res["ours"]["clocks"]}
@@ -507,7 +530,7 @@ def main():
         import datetime
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     d = make_inputs(w, seed=w.seed + rank)
     dev = torch.device("cuda", local)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -584,15 +607,18 @@ def main():
     gemm_ms = sum(phases[k][0] for k in gemm_phases)
     gemm_launches = sum(phases[k][1] for k in gemm_phases)
     achieved = w.useful_flops * args.steps / (gemm_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    # the timed region is well under the seconds-long loop the sustained figure
+    # was measured over, so the kernel is scored against the burst peak; the
+    # sustained fraction is reported beside it
+    peak = peaks["bf16_tflops"]
     traffic = recorded_traffic(w.name)
     roof = {"kernel": "tc_gemm_pair_kernel (logits, grad_X, grad_W launches)", "bound": "tensor",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic["bytes_per_launch"] if traffic else None,
             "traffic_source": traffic["source"] if traffic else "no capture of the current kernel source",
             "algorithmic_flops_per_launch": w.useful_flops * args.steps / max(gemm_launches, 1),
-            "peak_kind": f"{peaks['source']} sustained bf16 (the kernel runs inside a long step loop)",
-            "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+            "peak_kind": f"{peaks['source']} burst bf16 (timed region {ms / 1e3:.2f} s)",
+            "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
             "launches": gemm_launches, "avg_launch_ms": gemm_ms / max(gemm_launches, 1)}
     all_ms = sum(v[0] for v in phases.values())
 
@@ -668,8 +694,8 @@ def main():
                    "chunk_rows": st["chunk_rows"], "n_chunks": st["n_chunks"],
                    "grad_w_accum": args.grad_w_accum},
         "tflops": tflops,
-        "frac_of_bf16_peak": tflops / peaks["bf16_tflops_sustained"],
-        "frac_of_bf16_burst_peak": tflops / peaks["bf16_tflops"],
+        "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+        "frac_of_bf16_sustained_peak": tflops / peaks["bf16_tflops_sustained"],
         "peak_workspace_bytes": st["workspace_bytes"],
         "peak_extra_torch_bytes": peak_extra_torch,
         "materialized_logits_bytes": st["materialized_logits_bytes"],

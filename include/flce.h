@@ -111,7 +111,9 @@ typedef enum {
 #define FLCE_FLAG_FROM_KEPT 0x8
 
 typedef struct {
-  int64_t chunk_rows;            /* rows per chunk; 0 = chosen from workspace_limit_bytes.
+  int64_t chunk_rows;            /* rows per chunk; 0 = the environment variable
+                                    FLCE_CHUNK_ROWS if it holds a positive integer, else
+                                    chosen from workspace_limit_bytes.
                                     Rounded up to a multiple of 128. */
   int64_t workspace_limit_bytes; /* chunk store budget; 0 = at most 512 MiB but at least 2048
                                     rows, and at most half the rows, so two or more chunks
@@ -233,9 +235,12 @@ FLCE_API flce_status flce_cross_entropy(const flce_tensor* logits, const flce_te
  * captured around them, inside a host that owns all device memory through its
  * own allocator, or in a loop where an allocation and the synchronisation it
  * may bring are not allowed).
- *   Arguments and results are those of flce_cross_entropy (opt is not taken:
- *   the mean uses this call's own count of non-ignored rows). The caller still
- *   provides logits, target, loss and grad_logits (which may be the logits).
+ *   Arguments and results are those of flce_cross_entropy, with two
+ *   differences: opt is not taken (the mean uses this call's own count of
+ *   non-ignored rows), and reduction must be FLCE_MEAN or FLCE_SUM (FLCE_NONE
+ *   returns FLCE_ERR_INVALID_ARG: per-row losses come from flce_cross_entropy).
+ *   The caller still provides logits, target, loss and grad_logits (which may
+ *   be the logits).
  *   Scratch comes from one fixed array of 8 MiB in device memory that every
  *   GPU loading the library holds until the process exits. It needs about
  *   8 * ceil(V / 1024) + 12 bytes per row (round BT up to a multiple of 32
@@ -263,6 +268,23 @@ FLCE_API flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const
 FLCE_API flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N,
                            int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn_major,
                            int32_t b_mn_major, flce_stream_t stream);
+
+/*
+ * Upstream gradient: t *= *scale in place, on `stream`. The loss module of
+ * "Liger-Kernel 項目詳細介紹" (使用方法 > 3. 低級 API 方式) is used as
+ * loss = loss_fn(weight, input, target); loss.backward(). The fused call has
+ * already produced the gradients for an upstream gradient of 1 during the
+ * forward pass; backward multiplies them by the upstream gradient, which lives
+ * in device memory. So the comparison with 1 is made on the device: the host
+ * never waits for the value, and when it is exactly 1 no element of t is read
+ * or written.
+ *   t      bf16 or f32, ndim 0, 1 or 2 (unit inner stride; row pitch stride[0]);
+ *          DEVICE memory owned by the caller, modified in place
+ *   scale  DEVICE pointer to one f32
+ * Returns FLCE_ERR_INVALID_ARG for null pointers or a bad layout (nothing is
+ * enqueued then) and FLCE_ERR_UNSUPPORTED_DTYPE for other dtypes.
+ */
+FLCE_API flce_status flce_scale_grad(flce_tensor* t, const float* scale, flce_stream_t stream);
 
 /*
  * Waits for `stream`, then returns the device error word of the current

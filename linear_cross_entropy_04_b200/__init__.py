@@ -7,7 +7,7 @@ the library; the first call does, and raises if it is missing.
 """
 
 __all__ = [
-    "fused_linear_cross_entropy", "cross_entropy", "count_valid", "gemm_bf16", "plan",
+    "fused_linear_cross_entropy", "cross_entropy", "count_valid", "gemm_bf16", "plan", "scale_grad_",
     "device_error", "phase_times", "FusedLinearCrossEntropyLoss",
     "forward_keep", "backward_from_kept", "keep_workspace_bytes", "KeptLogits",
 ]

@@ -83,6 +83,7 @@ _SIGS = {
     "flce_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]),
+    "flce_scale_grad": (ctypes.c_int, [_P(FlceTensor), ctypes.c_void_p, ctypes.c_void_p]),
     "flce_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _P(ctypes.c_uint32)]),
     "flce_phase_times": (ctypes.c_int, [_P(ctypes.c_double), _P(ctypes.c_int32), ctypes.c_int32,
                                         ctypes.c_int32]),

@@ -249,6 +249,17 @@ def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, M: int, N: int, K: int, a_mn_ma
     return C
 
 
+def scale_grad_(t: torch.Tensor, scale: torch.Tensor, stream=None) -> torch.Tensor:
+    """t *= scale in place, scale a one-element fp32 device tensor; nothing is
+    read or written when it is exactly 1, and the host never waits for it."""
+    if scale.dtype != torch.float32 or scale.device != t.device or scale.numel() != 1:
+        scale = scale.to(device=t.device, dtype=torch.float32)
+    scale = scale.reshape(())
+    tt = B.tensor(t)
+    B.check(B.lib().flce_scale_grad(ctypes.byref(tt), B.ptr(scale), B.stream_handle(stream)), "flce_scale_grad")
+    return t
+
+
 def plan(BT: int, H: int, V: int, dtype: str = "bf16", want_grad_W: bool = True,
          chunk_rows: int = 0, workspace_limit_bytes: int = 0, grad_w_accum: str = "output") -> dict:
     """Chunk rows, chunk count and workspace bytes for a shape (host only)."""
@@ -277,7 +288,10 @@ def phase_times(reset: bool = True) -> dict:
 
 class _FLCEFunction(torch.autograd.Function):
     """'mean' / 'sum': the forward computes the loss and both gradients at
-    once, and backward hands them back scaled by the upstream gradient.
+    once, and backward hands them back scaled by the upstream gradient, in
+    place and on the device (flce_scale_grad), so backward never waits for the
+    GPU. The saved gradients are handed out once: a second backward through
+    the same graph raises instead of scaling them a second time.
     'none': the forward computes only the per-row losses; backward runs the
     fused path again with the per-row upstream gradient (row_grad), so the
     logits GEMM is done twice in exchange for never storing dlogits. With
@@ -327,11 +341,14 @@ class _FLCEFunction(torch.autograd.Function):
                                                        row_grad=grad_out.reshape(-1), want_grad_X=want_x,
                                                        want_grad_W=want_w, grad_w_accum=ctx.grad_w_accum)
             return gW, (gX.reshape(ctx.shape) if gX is not None else None), None, None, None, None, None
+        if getattr(ctx, "consumed", False):
+            raise RuntimeError("fused linear cross-entropy: its gradients were computed in the forward pass and "
+                               "were already scaled in place by an earlier backward through this graph")
+        ctx.consumed = True
         gX, gW = ctx.saved_tensors
         hx, hw = ctx.has
-        one = grad_out.numel() == 1 and bool(grad_out == 1)
-        dX = (gX if one else gX * grad_out.to(gX.dtype)).reshape(ctx.shape) if hx else None
-        dW = (gW if one else gW * grad_out.to(gW.dtype)) if hw else None
+        dX = scale_grad_(gX, grad_out).reshape(ctx.shape) if hx else None
+        dW = scale_grad_(gW, grad_out) if hw else None
         return dW, dX, None, None, None, None, None
 
 

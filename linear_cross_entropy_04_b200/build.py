@@ -7,6 +7,7 @@ linked statically and the driver's cuTensorMapEncodeTiled is looked up at run
 time, so the library also loads on a host without a GPU or driver (its
 argument checks and planning then work; compute calls need a B200).
 """
+import glob
 import os
 import shutil
 import subprocess
@@ -16,8 +17,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "flce.cu")
 OUT = os.path.join(PKG, "libflce.so")
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("flce.cu", "tc_gemm.cuh", "aux_kernels.cuh", "ptx.cuh")] + [
-    os.path.join(ROOT, "include", "flce.h")]
+
+def deps():
+    """Every source the library is compiled from: all of csrc/ and the public headers."""
+    return sorted(glob.glob(os.path.join(PKG, "csrc", "*")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def nvcc_path():
@@ -41,7 +44,7 @@ def up_to_date():
     if not os.path.exists(OUT):
         return False
     t = os.path.getmtime(OUT)
-    return all(os.path.getmtime(d) <= t for d in DEPS)
+    return all(os.path.getmtime(d) <= t for d in deps())
 
 
 def build(force=False, verbose=False, out=None, defines=()):

@@ -10,6 +10,9 @@
 //   factor_kernel        combine's factor step alone, for gradients taken from
 //                        a kept forward pass (FLCE_FLAG_FROM_KEPT)
 //   finalize_loss_kernel fixed-order sum of the per-row losses, times 1/N or 1
+//   scale_grad_kernel    gradients from the forward pass times the upstream
+//                        gradient (a device scalar), in place; no memory
+//                        traffic when that scalar is 1
 //   ce_row_cluster_kernel logits given, bf16: one cluster of CTAs per row, z
 //                        read once and dz written once
 //   ce_partials_kernel   logits given (f32, or rows too long for a cluster):
@@ -579,6 +582,41 @@ __global__ void __launch_bounds__(1024) finalize_loss_kernel(const float* __rest
       } else {
         *loss = (float)acc;
       }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ upstream gradient
+// p[r, c] *= *scale for a rows x cols matrix with row pitch ld (elements), in
+// 16-byte vectors (VEC elements; cols, ld and p aligned to them) or, VEC = 1,
+// one element at a time. The scale is read on the device, so the caller need
+// not wait for it; when it is exactly 1 every block returns before touching p.
+template <typename T, int VEC>
+__global__ void __launch_bounds__(256) scale_grad_kernel(T* __restrict__ p, int64_t rows, int64_t cols, int64_t ld,
+                                                         const float* __restrict__ scale) {
+  const float f = *scale;
+  if (f == 1.f) return;
+  const int64_t vpr = cols / VEC;  // vectors per row
+  const int64_t n = rows * vpr;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / vpr, c = (i - r * vpr) * VEC;
+    T* q = p + r * ld + c;
+    if constexpr (VEC == 1) {
+      if constexpr (sizeof(T) == 2) *q = __float2bfloat16_rn(__bfloat162float(*q) * f);
+      else *q = *q * f;
+    } else if constexpr (sizeof(T) == 2) {
+      uint4 v = *reinterpret_cast<const uint4*>(q);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 x = unpack_bf16x2(w[k]);
+        w[k] = pack_bf16x2(x.x * f, x.y * f);
+      }
+      *reinterpret_cast<uint4*>(q) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      float4 v = *reinterpret_cast<const float4*>(q);
+      v.x *= f; v.y *= f; v.z *= f; v.w *= f;
+      *reinterpret_cast<float4*>(q) = v;
     }
   }
 }

@@ -223,6 +223,18 @@ int64_t gradx_partial_elems(int64_t BT, int64_t H, int64_t V, int64_t chunk) {
   return best;
 }
 
+// FLCE_CHUNK_ROWS=<n> sets the chunk rows of calls whose options leave
+// chunk_rows at 0 (rounded up to a multiple of 128, like the option).
+// Unset, empty, non-numeric or non-positive values leave the default plan.
+int64_t env_chunk_rows() {
+  const char* s = std::getenv("FLCE_CHUNK_ROWS");
+  if (!s || !*s) return 0;
+  char* end = nullptr;
+  const long long v = std::strtoll(s, &end, 10);
+  if (end == s || *end != '\0' || v <= 0) return 0;
+  return round_up(std::min<int64_t>(v, kMaxChunk), 128);
+}
+
 struct Plan {
   int64_t BT, H, V;
   int32_t dtype;
@@ -248,7 +260,7 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
   p->ntile = ceil_div(V, p->tile_w);
   p->lde = round_up(V, 64);
   const int64_t per_row = p->lde * esz + p->ntile * 8 + 4;
-  int64_t chunk = opt && opt->chunk_rows > 0 ? round_up(opt->chunk_rows, 128) : 0;
+  int64_t chunk = opt && opt->chunk_rows > 0 ? round_up(opt->chunk_rows, 128) : env_chunk_rows();
   const int64_t bt_r = std::max<int64_t>(round_up(std::max<int64_t>(BT, 1), 128), 128);
   p->keep = opt && (opt->flags & (FLCE_FLAG_KEEP_LOGITS | FLCE_FLAG_FROM_KEPT));
   if (p->keep) {
@@ -1175,6 +1187,47 @@ flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, in
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
   if (env_debug() && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
+
+flce_status flce_scale_grad(flce_tensor* t, const float* scale, flce_stream_t stream) {
+  if (!t || !scale) return FLCE_ERR_INVALID_ARG;
+  if (t->dtype != FLCE_BF16 && t->dtype != FLCE_F32) return FLCE_ERR_UNSUPPORTED_DTYPE;
+  if (t->ndim < 0 || t->ndim > 2) return FLCE_ERR_INVALID_ARG;
+  int64_t rows = 1, cols = 1, ld = 1;
+  if (t->ndim == 1) {
+    cols = t->shape[0];
+    if (cols < 0 || (cols > 1 && t->stride[0] != 1)) return FLCE_ERR_INVALID_ARG;
+    ld = cols;
+  } else if (t->ndim == 2) {
+    rows = t->shape[0];
+    cols = t->shape[1];
+    if (rows < 0 || cols < 0 || (cols > 1 && t->stride[1] != 1) || (rows > 1 && t->stride[0] < cols))
+      return FLCE_ERR_INVALID_ARG;
+    ld = rows > 1 ? t->stride[0] : cols;
+  }
+  if (rows == 0 || cols == 0) return FLCE_OK;
+  if (!t->data) return FLCE_ERR_INVALID_ARG;
+  DeviceCtx* dev = nullptr;
+  const flce_status st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int esz = dtype_size(t->dtype);
+  const int vec = 16 / esz;
+  const bool vector = cols % vec == 0 && ld % vec == 0 && is_aligned(t->data, 16);
+  const int64_t units = rows * (vector ? cols / vec : cols);
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(units, 256), 8ll * dev->sms));
+  if (t->dtype == FLCE_BF16) {
+    __nv_bfloat16* p = static_cast<__nv_bfloat16*>(t->data);
+    if (vector) scale_grad_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, s>>>(p, rows, cols, ld, scale);
+    else scale_grad_kernel<__nv_bfloat16, 1><<<blocks, 256, 0, s>>>(p, rows, cols, ld, scale);
+  } else {
+    float* p = static_cast<float*>(t->data);
+    if (vector) scale_grad_kernel<float, 4><<<blocks, 256, 0, s>>>(p, rows, cols, ld, scale);
+    else scale_grad_kernel<float, 1><<<blocks, 256, 0, s>>>(p, rows, cols, ld, scale);
+  }
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (env_debug() && cudaStreamSynchronize(s) != cudaSuccess) return FLCE_ERR_CUDA;
   return FLCE_OK;
 }
 

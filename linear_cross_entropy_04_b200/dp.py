@@ -97,7 +97,11 @@ def dp_fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torc
     supply them (buf, peers, shard_rows, rank, barrier()); by default they are
     symmetric-memory buffers.
     Every rank takes the same collective steps in the same order.
+    reduction 'none' is refused (ValueError) before any collective: its
+    per-row losses stay with their rank and there is no global loss to reduce.
     """
+    if reduction not in ("mean", "sum"):
+        raise ValueError(f"data-parallel reduction must be 'mean' or 'sum', not {reduction!r}")
     if fused_grad_W:
         return _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, shards, count_fn,
                                 flce_fn, **kw)

@@ -129,6 +129,14 @@ def test_other_entry_points_validate(lib):
                                   None) == 1
     assert lib.flce_get_device_error(None, None) == 1
     assert lib.flce_phase_times(None, None, -1, 0) == 1
+    g = _t(FAKE, B.BF16, (4, 100))
+    assert lib.flce_scale_grad(None, FAKE, None) == 1                    # no tensor
+    assert lib.flce_scale_grad(ctypes.byref(g), None, None) == 1         # no scale
+    assert lib.flce_scale_grad(ctypes.byref(tg), FAKE, None) == 2        # int64 is not a gradient
+    bad = _t(FAKE, B.BF16, (4, 100), stride=(50, 1))                     # rows overlap
+    assert lib.flce_scale_grad(ctypes.byref(bad), FAKE, None) == 1
+    empty = _t(None, B.F32, (0, 8))
+    assert lib.flce_scale_grad(ctypes.byref(empty), FAKE, None) == 0     # nothing to scale, no device needed
 
 
 def test_plan_is_host_only_and_bounded(lib):
@@ -264,3 +272,43 @@ def test_python_api_rejects_bad_option_strings():
         api.forward_keep(X, W, t, reduction="mean_")
     with pytest.raises(ValueError, match="grad_w_accum"):
         api.plan(4, 8, 10, grad_w_accum="fp16")
+
+
+def test_build_dependencies_cover_every_source(tmp_path, monkeypatch):
+    """Every file under csrc/ and every public header counts for up_to_date():
+    touching any one of them makes the built library stale."""
+    srcs = set(os.listdir(os.path.join(build_mod.PKG, "csrc")))
+    deps = build_mod.deps()
+    assert {os.path.basename(d) for d in deps if os.sep + "csrc" + os.sep in d} == srcs
+    assert HEADER in deps
+    # a fake library newer than every source is up to date until one source is newer
+    fake = tmp_path / "libflce.so"
+    fake.write_bytes(b"")
+    newest = max(os.path.getmtime(d) for d in deps)
+    os.utime(fake, (newest + 10, newest + 10))
+    monkeypatch.setattr(build_mod, "OUT", str(fake))
+    assert build_mod.up_to_date()
+    os.utime(fake, (newest - 1, newest - 1))
+    assert not build_mod.up_to_date()
+
+
+def test_chunk_rows_environment_override(lib, monkeypatch):
+    """FLCE_CHUNK_ROWS sets the chunk rows when the options leave them at 0; an
+    explicit option wins, and values that are not positive integers are ignored."""
+    def plan(opt_rows=0):
+        o = B.FlceOptions()
+        lib.flce_options_init(ctypes.byref(o))
+        o.chunk_rows = opt_rows
+        st = B.FlceStats()
+        assert lib.flce_plan(4096, 4096, 128256, B.BF16, 1, ctypes.byref(o), ctypes.byref(st)) == 0
+        return st.chunk_rows, st.n_chunks
+
+    monkeypatch.delenv("FLCE_CHUNK_ROWS", raising=False)
+    default = plan()
+    assert default == (2048, 2)
+    monkeypatch.setenv("FLCE_CHUNK_ROWS", "1000")
+    assert plan() == (1024, 4)          # rounded up to 128
+    assert plan(opt_rows=512) == (512, 8)
+    for bad in ("", "abc", "-5", "0", "12x"):
+        monkeypatch.setenv("FLCE_CHUNK_ROWS", bad)
+        assert plan() == default, bad

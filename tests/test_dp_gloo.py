@@ -168,6 +168,18 @@ def test_shard_sizes():
         assert sum(owned_rows(V, S, r) for r in range(world)) == V
 
 
+def test_none_reduction_is_refused_before_any_collective():
+    """'none' has no global loss; the call fails at once, with no process group at all."""
+    import torch
+
+    from linear_cross_entropy_04_b200.dp import dp_fused_linear_cross_entropy
+
+    X, W, t = torch.zeros(4, 8), torch.zeros(10, 8), torch.zeros(4, dtype=torch.int64)
+    for fused in (False, True):
+        with pytest.raises(ValueError, match="reduction"):
+            dp_fused_linear_cross_entropy(X, W, t, reduction="none", fused_grad_W=fused)
+
+
 class _CpuShards:
     """Shards in shared memory. The emulated device call adds into them from a
     background thread (device work is asynchronous); barrier() first waits for

@@ -205,6 +205,50 @@ def test_module_autograd_matches_oracle():
     assert_grad_close(W.grad, 2.5 * ref["grad_W"], "bf16", "module grad_W")
 
 
+def test_module_backward_does_not_wait_for_the_gpu():
+    """backward applies the upstream gradient on the device: with the stream kept
+    busy by a long spin kernel, backward returns before that kernel ends, and the
+    gradients still come out scaled (1 leaves them untouched, 0.5 halves them)."""
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
+    ref = oracle.flce(d["X"], d["W"], d["target"])
+    for factor in (1.0, 0.5):
+        X, W, t = to_dev(d)
+        X.requires_grad_(True)
+        W.requires_grad_(True)
+        loss = L().FusedLinearCrossEntropyLoss()(W, X, t)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000_000)  # about a second of spinning ahead of backward's work
+        (loss * factor).backward()
+        busy = not torch.cuda.current_stream().query()
+        torch.cuda.synchronize()
+        assert busy, "backward waited for the GPU"
+        assert_grad_close(X.grad, factor * ref["grad_X"], "bf16", f"grad_X x{factor}")
+        assert_grad_close(W.grad, factor * ref["grad_W"], "bf16", f"grad_W x{factor}")
+        with pytest.raises(RuntimeError, match="already scaled"):
+            loss2 = L().FusedLinearCrossEntropyLoss()(W.detach().requires_grad_(True), X.detach(), t)
+            loss2.backward(retain_graph=True)
+            loss2.backward()
+
+
+def test_scale_grad_layouts():
+    """flce_scale_grad on vector and element paths, strided rows, both dtypes."""
+    g = torch.Generator(device="cuda").manual_seed(3)
+    for dt in (torch.bfloat16, torch.float32):
+        for shape, cols in (((300, 264), 264), ((64, 101), 101), ((7,), None)):
+            base = torch.randn(*shape, generator=g, device="cuda").to(dt)
+            if cols == 264:
+                big = torch.randn(300, 272, generator=g, device="cuda").to(dt)
+                base = big[:, :264]  # row pitch 272
+            ref = base.float() * 0.3
+            s = torch.tensor(0.3, device="cuda")
+            L().scale_grad_(base, s)
+            tol = 2 ** -8 if dt == torch.bfloat16 else 1e-6
+            assert torch.allclose(base.float(), ref, rtol=tol, atol=0)
+            before = base.clone()
+            L().scale_grad_(base, torch.tensor(1.0, device="cuda"))
+            assert torch.equal(base, before)
+
+
 def test_host_buffers_end_to_end():
     d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
     X = torch.from_numpy(d["X"]).to(torch.bfloat16).pin_memory()
