@@ -115,7 +115,7 @@ def make_inputs(w: Workload, BT: Optional[int] = None, H: Optional[int] = None,
     target = draw_targets(rng, BT, V, w.targets, w.ignore_frac, w.zipf_s)
     return {
         "X": round_to_dtype(X, w.dtype),
-        "W": round_to_dtype(W, w.dtype),
+        "W": W if w_zero else round_to_dtype(W, w.dtype),  # zeros are exact in every dtype
         "target": target,
         "dtype": w.dtype,
         "BT": BT, "H": H, "V": V,
