@@ -54,6 +54,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--chunk-rows", type=int, default=0)
     ap.add_argument("--grad-w-accum", default="output", choices=["output", "fp32"])
+    ap.add_argument("--schedule", default="stored", choices=["stored", "recompute"],
+                    help="stored: row chunks keep their logits store (6*BT*H*V tensor FLOPs, the default); "
+                         "recompute: vocabulary chunks, logits rebuilt after an lse pass (8*BT*H*V)")
+    ap.add_argument("--workspace-limit-mib", type=int, default=0, help="chunk store budget (0: the library default)")
     ap.add_argument("--dp-fused-grad-w", action="store_true",
                     help="N > 1: reduce-scatter grad_W inside the grad_W GEMM over NVLink (symmetric memory) "
                          "instead of an NCCL all-reduce after it")
@@ -541,7 +545,8 @@ def main():
     gX = torch.empty_like(X)
     gW = torch.empty_like(W)
     nvalid = torch.empty((), dtype=torch.int64, device=dev)
-    kw = dict(chunk_rows=args.chunk_rows, grad_w_accum=args.grad_w_accum)
+    kw = dict(chunk_rows=args.chunk_rows, grad_w_accum=args.grad_w_accum, schedule=args.schedule,
+              workspace_limit_bytes=args.workspace_limit_mib << 20)
 
     from linear_cross_entropy_04_b200.dp import dp_fused_linear_cross_entropy
 
@@ -619,7 +624,9 @@ def main():
             "algorithmic_flops_per_launch": w.useful_flops * args.steps / max(gemm_launches, 1),
             "peak_kind": f"{peaks['source']} burst bf16 (timed region {ms / 1e3:.2f} s)",
             "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
-            "launches": gemm_launches, "avg_launch_ms": gemm_ms / max(gemm_launches, 1)}
+            "launches": gemm_launches, "avg_launch_ms": gemm_ms / max(gemm_launches, 1),
+            # the recompute schedule executes 8*BT*H*V tensor FLOPs for the 6 that count
+            "executed_tflops": achieved * (8.0 if args.schedule == "recompute" else 6.0) / 6.0}
     all_ms = sum(v[0] for v in phases.values())
 
     # end to end through the public API with host buffers: every step copies
@@ -692,7 +699,7 @@ def main():
                                        else "NCCL all-reduce") if world > 1 else None,
                    "l2": "inputs larger than L2 (W alone is %.2f GB)" % (w.V * w.H * 2 / 1e9),
                    "chunk_rows": st["chunk_rows"], "n_chunks": st["n_chunks"],
-                   "grad_w_accum": args.grad_w_accum},
+                   "grad_w_accum": args.grad_w_accum, "schedule": args.schedule},
         "tflops": tflops,
         "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
         "frac_of_bf16_sustained_peak": tflops / peaks["bf16_tflops_sustained"],

@@ -109,6 +109,25 @@ typedef enum {
  * pairs; keeping the batch's store is the general form of that on one chunk. */
 #define FLCE_FLAG_KEEP_LOGITS 0x4
 #define FLCE_FLAG_FROM_KEPT 0x8
+/* grad_W shards (below): route every chunk's grad_W boxes to their owners
+ * instead of only the last chunk's. No local [V, H] partial sum is kept, at the
+ * price of n_chunks times the exchanged bytes. */
+#define FLCE_FLAG_ROUTE_EVERY_CHUNK 0x10
+/* The recompute schedule (bf16 only; not with the two-phase flags or grad_W
+ * shards). The pages' chunked method (技術原理 > 分塊計算 of "Liger-Kernel
+ * 項目詳細介紹") bounds memory by computing the logits a piece at a time; this
+ * schedule takes the pieces over the vocabulary instead of the rows. A first
+ * pass computes every row's logsumexp with nothing stored; a second pass, per
+ * chunk of Vc vocabulary columns, rebuilds the logits of all rows over the
+ * chunk by GEMM, writes dz into a [BT, Vc] bf16 store, adds dz W_c into grad_X
+ * (in bf16, one rounding per chunk after the first) and writes the chunk's rows
+ * of grad_W = dz^T X complete. 8 * BT * H * V tensor FLOPs instead of 6; in
+ * exchange the store can be as small as BT * 256 * 2 bytes. With this flag,
+ * chunk_rows (if > 0) is the vocabulary columns per chunk (rounded up to 256),
+ * else Vc comes from workspace_limit_bytes (default 512 MiB) over BT rows; the
+ * stats' chunk_rows / n_chunks then describe vocabulary chunks. grad_w_accum
+ * has no effect: every grad_W row is produced once. */
+#define FLCE_FLAG_RECOMPUTE 0x20
 
 typedef struct {
   int64_t chunk_rows;            /* rows per chunk; 0 = the environment variable
@@ -133,10 +152,14 @@ typedef struct {
   /* grad_W scattered to shards (data parallelism): shard k (< n_shards <= 8) owns grad_W rows
      [k * shard_rows, (k+1) * shard_rows), stored bf16 [rows, H] with row pitch grad_w_shard_ld
      at grad_w_shards[k] (a HOST array of device pointers; a shard may live on a peer GPU, mapped
-     into this one). Every grad_W tile is ADDED into its owner's shard as it is produced (a TMA
-     reduce-add, done in the owner's L2, over NVLink for a peer), for every chunk. So the caller
-     zeroes each shard and orders that before any rank's call, and orders every rank's call
-     before reading a shard. Requires the bf16 path, grad_W == NULL, shard_rows % 32 == 0 and
+     into this one). The chunks before the last accumulate grad_W locally, in a bf16 [V, H]
+     region of the workspace (flce_plan counts it); the last chunk's grad_W GEMM adds each of its
+     output boxes, plus the same box of that local sum, into the owner's shard as it is produced
+     (a TMA reduce-add, done in the owner's L2, over NVLink for a peer). So each rank sends
+     V * H * 2 bytes whatever the chunk count, (P - 1) / P of them to peers.
+     FLCE_FLAG_ROUTE_EVERY_CHUNK routes every chunk's boxes instead (no local sum).
+     The caller zeroes each shard and orders that before any rank's call, and orders every rank's
+     call before reading a shard. Requires the bf16 path, grad_W == NULL, shard_rows % 32 == 0 and
      n_shards * shard_rows >= V. Additions from several callers land in unspecified order. */
   void* const* grad_w_shards;
   int32_t n_shards;
@@ -268,6 +291,24 @@ FLCE_API flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const
 FLCE_API flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N,
                            int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn_major,
                            int32_t b_mn_major, flce_stream_t stream);
+
+/*
+ * Test of the engine's failure path; the paper has no counterpart. The plain
+ * GEMM of flce_gemm_bf16 (both operands K-major) on the CTA-pair engine, with
+ * one change: every pair's MMA issuer, before its output tile number
+ * stall_tile (0 = its first), waits on a barrier that nothing arrives on. That
+ * wait is bounded like every wait in the library, so it runs out after the
+ * library's wait limit (about 2 s): the kernel sets FLCE_DEVERR_TIMEOUT in the
+ * device error word, abandons its remaining tiles, waits for the loads and
+ * tensor-core work it has in flight, frees its tensor memory and returns. The
+ * caller reads the status with flce_get_device_error; C is left partly written.
+ * The context stays usable: later calls run normally. Returns FLCE_ERR_INVALID_ARG
+ * for the arguments flce_gemm_bf16 refuses, a negative stall_tile, or when the
+ * single-CTA engine is selected (FLCE_ENGINE=1sm).
+ */
+FLCE_API flce_status flce_gemm_bf16_wait_test(const void* A, const void* B, float* C, int64_t M, int64_t N,
+                                              int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t stall_tile,
+                                              flce_stream_t stream);
 
 /*
  * Upstream gradient: t *= *scale in place, on `stream`. The loss module of

@@ -19,6 +19,7 @@ LIB_PATH = os.environ.get("FLCE_LIBRARY") or os.path.join(PKG, "libflce.so")
 F32, BF16, I64 = 0, 1, 2
 MEAN, SUM, NONE = 0, 1, 2
 FLAG_SYNC_CHECK, FLAG_TIME_PHASES, FLAG_KEEP_LOGITS, FLAG_FROM_KEPT = 0x1, 0x2, 0x4, 0x8
+FLAG_ROUTE_EVERY_CHUNK, FLAG_RECOMPUTE = 0x10, 0x20
 GRADW_ACCUM_OUTPUT, GRADW_ACCUM_FP32 = 0, 1
 DEVERR_TARGET_RANGE, DEVERR_TIMEOUT = 0x1, 0x2
 NUM_PHASES = 6
@@ -83,6 +84,9 @@ _SIGS = {
     "flce_gemm_bf16": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]),
+    "flce_gemm_bf16_wait_test": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p]),
     "flce_scale_grad": (ctypes.c_int, [_P(FlceTensor), ctypes.c_void_p, ctypes.c_void_p]),
     "flce_get_device_error": (ctypes.c_int, [ctypes.c_void_p, _P(ctypes.c_uint32)]),
     "flce_phase_times": (ctypes.c_int, [_P(ctypes.c_double), _P(ctypes.c_int32), ctypes.c_int32,

@@ -18,9 +18,18 @@ _RED = {"mean": B.MEAN, "sum": B.SUM, "none": B.NONE}
 _ACC = {"output": B.GRADW_ACCUM_OUTPUT, "fp32": B.GRADW_ACCUM_FP32}
 
 
+_SCHED = {"stored": 0, "recompute": B.FLAG_RECOMPUTE}
+
+
 def _check_reduction(reduction):
     if reduction not in _RED:
         raise ValueError(f"reduction must be one of {sorted(_RED)}, not {reduction!r}")
+
+
+def _schedule_flag(schedule):
+    if schedule not in _SCHED:
+        raise ValueError(f"schedule must be one of {sorted(_SCHED)}, not {schedule!r}")
+    return _SCHED[schedule]
 
 
 def _options(chunk_rows=0, workspace_limit_bytes=0, grad_w_accum="output", flags=0,
@@ -50,7 +59,7 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                grad_w_accum: str = "output", n_valid: Optional[torch.Tensor] = None,
                                row_loss: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                                row_grad: Optional[torch.Tensor] = None, grad_w_shards=None,
-                               shard_rows: int = 0,
+                               shard_rows: int = 0, schedule: str = "stored",
                                flags: int = 0, stream=None, out=None, host_out=None,
                                return_stats: bool = False):
     """Loss, grad_X and grad_W of cross-entropy over X W^T in one call.
@@ -68,9 +77,15 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     host_out = (loss, grad_X, grad_W) pinned host tensors receive them then.
     out = (loss, grad_X, grad_W) preallocated device tensors may be given.
     The library's workspace is taken from torch's caching allocator.
+    schedule 'stored' (default) chunks the rows and keeps each chunk's logits
+    store (6*BT*H*V tensor FLOPs); 'recompute' chunks the vocabulary, computes
+    every row's logsumexp first and rebuilds the logits per vocabulary chunk
+    (8*BT*H*V tensor FLOPs; the store is [BT, chunk_rows] with chunk_rows read
+    as vocabulary columns, or sized from workspace_limit_bytes).
     Returns (loss [scalar fp32], grad_X or None, grad_W or None[, stats]).
     """
     _check_reduction(reduction)
+    flags = int(flags) | _schedule_flag(schedule)
     host = not X.is_cuda
     if host:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -261,9 +276,11 @@ def scale_grad_(t: torch.Tensor, scale: torch.Tensor, stream=None) -> torch.Tens
 
 
 def plan(BT: int, H: int, V: int, dtype: str = "bf16", want_grad_W: bool = True,
-         chunk_rows: int = 0, workspace_limit_bytes: int = 0, grad_w_accum: str = "output") -> dict:
-    """Chunk rows, chunk count and workspace bytes for a shape (host only)."""
-    o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum)
+         chunk_rows: int = 0, workspace_limit_bytes: int = 0, grad_w_accum: str = "output",
+         schedule: str = "stored") -> dict:
+    """Chunk rows (vocabulary columns for schedule 'recompute'), chunk count and
+    workspace bytes for a shape (host only)."""
+    o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags=_schedule_flag(schedule))
     st = B.FlceStats()
     rc = B.lib().flce_plan(BT, H, V, B.BF16 if dtype == "bf16" else B.F32, int(want_grad_W),
                            ctypes.byref(o), ctypes.byref(st))

@@ -23,6 +23,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/flce.h"
 #include "aux_kernels.cuh"
 #include "tc_gemm.cuh"
@@ -38,6 +40,7 @@ constexpr int kMaxDevices = 64;
 constexpr int64_t kDefaultLimit = 512ll << 20;
 constexpr int64_t kMaxChunk = 32768;
 constexpr int64_t kMinDefaultChunk = 2048;
+constexpr int64_t kRecomputeRowBlock = 4096;  // rows per logits launch in the recompute schedule's first pass
 
 struct DeviceCtx {
   bool init = false;
@@ -83,7 +86,9 @@ flce_status device_ctx(DeviceCtx** out) {
           cudaFuncSetAttribute(tc_gemm_pair_kernel<NoShards>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                T2_SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(tc_gemm_pair_kernel<ShardMaps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               T2_SMEM_BYTES) != cudaSuccess)
+                               T2_SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tc_gemm_pair_kernel<NoShards, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               T2W_SMEM_BYTES) != cudaSuccess)
         return FLCE_ERR_CUDA;
       {
         cudaLaunchConfig_t cfg;
@@ -241,9 +246,14 @@ struct Plan {
   int64_t chunk, n_chunks;
   int64_t tile_w;  // partial tile width (columns)
   int64_t ntile, lde, ldp;
-  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, off_xpart, off_lse, total;
+  size_t off_nvalid, off_rowloss, off_zt, off_pm, off_ps, off_e, off_facc, off_xpart, off_lse, off_gwl, total;
   bool keep;  // FLCE_FLAG_KEEP_LOGITS / FLCE_FLAG_FROM_KEPT: one chunk, lse kept in the workspace
   bool facc;
+  bool gw_local;  // grad_W shards: chunks before the last accumulate into a local bf16 [V, H]
+  // recompute schedule (FLCE_FLAG_RECOMPUTE): chunk = vocabulary columns per chunk, n_chunks =
+  // vocabulary chunks, the store is [BT, chunk]; the first pass takes rows in blocks of r1
+  bool recompute;
+  int64_t r1;
   int64_t xpart_elems;  // grad_X split-K partials (fp32 elements)
 };
 
@@ -263,6 +273,38 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
   int64_t chunk = opt && opt->chunk_rows > 0 ? round_up(opt->chunk_rows, 128) : env_chunk_rows();
   const int64_t bt_r = std::max<int64_t>(round_up(std::max<int64_t>(BT, 1), 128), 128);
   p->keep = opt && (opt->flags & (FLCE_FLAG_KEEP_LOGITS | FLCE_FLAG_FROM_KEPT));
+  p->recompute = opt && (opt->flags & FLCE_FLAG_RECOMPUTE);
+  p->gw_local = false;
+  p->r1 = 0;
+  if (p->recompute) {
+    if (dtype != FLCE_BF16) return FLCE_ERR_UNSUPPORTED_DTYPE;
+    if (p->keep || (opt->n_shards > 0)) return FLCE_ERR_INVALID_ARG;
+    // vocabulary columns per chunk: the option, else the store budget over all rows
+    int64_t vc = opt->chunk_rows > 0 ? round_up(opt->chunk_rows, 256) : 0;
+    if (vc == 0) {
+      const int64_t limit = opt->workspace_limit_bytes > 0 ? opt->workspace_limit_bytes : kDefaultLimit;
+      vc = (limit / (bt_r * 2)) / 256 * 256;
+    }
+    vc = std::max<int64_t>(256, std::min<int64_t>(vc, round_up(V, 256)));
+    p->chunk = vc;
+    p->n_chunks = BT > 0 ? ceil_div(V, vc) : 0;
+    p->lde = vc;
+    p->r1 = std::min<int64_t>(bt_r, kRecomputeRowBlock);
+    p->ldp = round_up(p->r1, 32);
+    p->facc = false;
+    p->xpart_elems = 0;
+    size_t o = 0;
+    p->off_nvalid = o; o = align256(o + 8);
+    p->off_rowloss = o; o = align256(o + (need_rowloss ? (size_t)std::max<int64_t>(BT, 1) * 4 : 0));
+    p->off_zt = o; o = align256(o + (size_t)p->r1 * 4);
+    p->off_pm = o; o = align256(o + (size_t)p->ntile * p->ldp * 4);
+    p->off_ps = o; o = align256(o + (size_t)p->ntile * p->ldp * 4);
+    p->off_e = o; o = align256(o + (size_t)std::max<int64_t>(BT, 1) * vc * 2);
+    p->off_lse = o; o = align256(o + (size_t)std::max<int64_t>(BT, 1) * 4);
+    p->off_facc = p->off_xpart = p->off_gwl = o;
+    p->total = o;
+    return FLCE_OK;
+  }
   if (p->keep) {
     // the whole batch is one chunk whose store outlives the call
     if (bt_r > kMaxChunk) return FLCE_ERR_INVALID_ARG;
@@ -302,6 +344,9 @@ flce_status make_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, bool want
   p->xpart_elems = dtype == FLCE_BF16 ? gradx_partial_elems(BT, H, V, chunk) : 0;
   p->off_xpart = o; o = align256(o + (size_t)p->xpart_elems * 4);
   p->off_lse = o; o = align256(o + (p->keep ? (size_t)chunk * 4 : 0));
+  p->gw_local = dtype == FLCE_BF16 && opt && opt->n_shards > 0 && !(opt->flags & FLCE_FLAG_ROUTE_EVERY_CHUNK) &&
+                p->n_chunks > 1;
+  p->off_gwl = o; o = align256(o + (p->gw_local ? (size_t)V * H * 2 : 0));
   p->total = o;
   return FLCE_OK;
 }
@@ -317,13 +362,34 @@ cudaEvent_t pool_event() {
   return e;
 }
 
-// Launch bookkeeping: optional phase events, launch-error checks, counts.
+// Names of the phases of flce_phase_times, also used for the NVTX ranges.
+const char* const kPhaseNames[FLCE_NUM_PHASES] = {"count_valid", "logits_gemm_softmax", "row_combine",
+                                                  "dlogits_inplace", "grad_gemms", "loss_reduce"};
+
+// NVTX range for the host-side span of a call or a phase launch (seen by
+// profilers that attach an NVTX tool; otherwise each push/pop is a no-op call).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// Launch bookkeeping: optional phase events, NVTX ranges, launch-error checks,
+// counts. `chunk` (or -1) names the row chunk in the phase's NVTX range.
 struct Launcher {
   cudaStream_t stream;
   bool timing, sync_check;
   int launches = 0;
+  int64_t chunk = -1;
   template <typename F>
   flce_status run(int phase, F&& f) {
+    char name[64];
+    if (chunk >= 0)
+      std::snprintf(name, sizeof(name), "flce %s chunk %lld", kPhaseNames[phase], (long long)chunk);
+    else
+      std::snprintf(name, sizeof(name), "flce %s", kPhaseNames[phase]);
+    const NvtxRange range(name);
     cudaEvent_t a = nullptr, b = nullptr;
     if (timing) {
       std::lock_guard<std::mutex> lk(g_mu);
@@ -407,6 +473,24 @@ bool ce_one_pass_enabled() {
   return !(s && std::strcmp(s, "multipass") == 0);
 }
 
+// Share of `units` workers kept busy over the waves of `tiles` equal tiles.
+double wave_efficiency(int64_t tiles, int64_t units) {
+  return (double)tiles / (double)(ceil_div(tiles, units) * units);
+}
+
+// grad_X on the pair engine's wide 256 x 512 tiles: when that keeps at least as
+// many pairs busy over its waves as 256 x 256 tiles would, and the narrow tiles
+// would not be run together with grad_W (which fills the pairs they leave idle).
+// FLCE_GRADX_TILE=wide|narrow forces the choice.
+bool gradx_wide(int64_t tiles_m, int64_t N, int64_t units) {
+  const char* s = std::getenv("FLCE_GRADX_TILE");
+  if (s && std::strcmp(s, "wide") == 0) return true;
+  if (s && std::strcmp(s, "narrow") == 0) return false;
+  const double en = wave_efficiency(tiles_m * ceil_div(N, 256), units);
+  const double ew = wave_efficiency(tiles_m * ceil_div(N, 512), units);
+  return ew >= en - 1e-9 && en >= 0.8;
+}
+
 bool grad_combined(int64_t gradx_tiles, int64_t units) {
   const char* s = std::getenv("FLCE_GRAD_LAUNCH");
   if (s && std::strcmp(s, "combined") == 0) return true;
@@ -441,9 +525,12 @@ bool make_out_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
   return make_tmap(m, base, cols, rows, ld * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// wide: the pair engine's 256 x 512 tiles (one problem, bf16 TMA-store epilogue,
+// tiles_n counted in 512-column tiles).
 void launch_tc(const Engine& eg, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
                const CUtensorMap& b1, const TcParams& prm, const DeviceCtx* dev, cudaStream_t stream,
-               const CUtensorMap* c0 = nullptr, const CUtensorMap* c1 = nullptr, const ShardMaps* shards = nullptr) {
+               const CUtensorMap* c0 = nullptr, const CUtensorMap* c1 = nullptr, const ShardMaps* shards = nullptr,
+               bool wide = false) {
   CUtensorMap zc;
   std::memset(&zc, 0, sizeof(zc));
   NoShards ns;
@@ -453,7 +540,10 @@ void launch_tc(const Engine& eg, const CUtensorMap& a0, const CUtensorMap& b0, c
   if (prm.nprob > 1) tiles += (int64_t)prm.prob[1].tiles_m * prm.prob[1].tiles_n;
   if (eg.pair) {
     const int pairs = (int)std::min<int64_t>(dev->pairs, tiles);
-    if (shards)
+    if (wide)
+      tc_gemm_pair_kernel<NoShards, true><<<2 * pairs, TC_THREADS, T2W_SMEM_BYTES, stream>>>(
+          a0, b0, a1, b1, c0 ? *c0 : zc, c1 ? *c1 : zc, ns, prm);
+    else if (shards)
       tc_gemm_pair_kernel<ShardMaps><<<2 * pairs, TC_THREADS, T2_SMEM_BYTES, stream>>>(
           a0, b0, a1, b1, c0 ? *c0 : zc, c1 ? *c1 : zc, *shards, prm);
     else
@@ -463,6 +553,141 @@ void launch_tc(const Engine& eg, const CUtensorMap& a0, const CUtensorMap& b0, c
     const int grid = (int)std::min<int64_t>(sms, tiles);
     tc_gemm_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, stream>>>(a0, b0, a1, b1, prm);
   }
+}
+
+// ------------------------------------------------------------------ recompute schedule
+// FLCE_FLAG_RECOMPUTE: the vocabulary-outer schedule. The first pass runs the
+// logits GEMM over row blocks with the online-softmax epilogue but stores
+// nothing, and the row combine keeps lse. The second pass takes the vocabulary
+// in chunks of Vc columns: the logits of all rows over the chunk are rebuilt
+// by GEMM and the epilogue writes dz = (softmax - onehot) * scale straight into
+// a [BT, Vc] store; then grad_X (+)= dz W_c (K = Vc; added into grad_X in L2
+// after the first chunk) and grad_W[chunk] = dz^T X (K = BT, complete in one
+// GEMM). 8 * BT * H * V tensor FLOPs instead of 6, for a store whose size the
+// caller picks down to BT * 256 * 2 bytes.
+flce_status run_recompute_passes(const flce_tensor* X, const flce_tensor* W, const int64_t* tgt,
+                                 int64_t ignore_index, int32_t reduction, flce_tensor* grad_X, flce_tensor* grad_W,
+                                 bool want_gx, bool want_gw, const Plan& pl, uint8_t* base, const int64_t* nvalid,
+                                 float* row_loss, const float* row_grad, float* lse_out, const Engine& eg,
+                                 const DeviceCtx* dev, cudaStream_t stream, Launcher& L) {
+  const int64_t BT = pl.BT, H = pl.H, V = pl.V;
+  const int64_t ldx = X->stride[0], ldw = W->stride[0];
+  const __nv_bfloat16* Xp = static_cast<const __nv_bfloat16*>(X->data);
+  const __nv_bfloat16* Wp = static_cast<const __nv_bfloat16*>(W->data);
+  float* zt = reinterpret_cast<float*>(base + pl.off_zt);
+  float* pm = reinterpret_cast<float*>(base + pl.off_pm);
+  float* ps = reinterpret_cast<float*>(base + pl.off_ps);
+  __nv_bfloat16* E = reinterpret_cast<__nv_bfloat16*>(base + pl.off_e);
+  float* lse = lse_out ? lse_out : reinterpret_cast<float*>(base + pl.off_lse);
+  CUtensorMap z;
+  std::memset(&z, 0, sizeof(z));
+  flce_status st = FLCE_OK;
+  // pass 1: row logsumexp and per-row losses, nothing stored
+  for (int64_t r0 = 0, blk = 0; r0 < BT; r0 += pl.r1, ++blk) {
+    L.chunk = blk;
+    const int rows = (int)std::min<int64_t>(pl.r1, BT - r0);
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, Xp + r0 * ldx, H, rows, ldx * 2, 64, 128) || !make_tmap(&tb, Wp, H, V, ldw * 2, 64, eg.b_box_rows))
+      return FLCE_ERR_CUDA;
+    TcParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.nprob = 1;
+    prm.prob[0] = make_problem(eg, rows, (int)V, (int)H, 0, 0, EPI_LOGITS, 1);
+    prm.lg.target = tgt + r0;
+    prm.lg.ignore_index = ignore_index;
+    prm.lg.V = V;
+    prm.lg.part_m = pm;
+    prm.lg.part_s = ps;
+    prm.lg.ldp = pl.ldp;
+    prm.lg.zt = zt;
+    prm.lg.store = 0;
+    prm.err = dev->err;
+    st = L.run(1, [&] { launch_tc(eg, ta, tb, z, z, prm, dev, stream, &z); });
+    if (st != FLCE_OK) return st;
+    CombineArgs a{tgt + r0, ignore_index, V, rows, (int)pl.ntile, pl.ldp, pm, ps, zt, row_loss + r0, lse + r0, nvalid,
+                  reduction, nullptr, 1};
+    st = L.run(2, [&] { combine_kernel<<<(unsigned)ceil_div(rows, 32), CB_THREADS, 0, stream>>>(a); });
+    if (st != FLCE_OK) return st;
+  }
+  if (!want_gx && !want_gw) return FLCE_OK;
+  // pass 2: per vocabulary chunk, dz by GEMM, then the two gradient contractions
+  const int64_t vc = pl.chunk;
+  for (int64_t c = 0; c < pl.n_chunks; ++c) {
+    L.chunk = c;
+    const int64_t v0 = c * vc;
+    const int cols = (int)std::min<int64_t>(vc, V - v0);
+    const __nv_bfloat16* Wc = Wp + v0 * ldw;
+    {
+      CUtensorMap ta, tb, te;
+      if (!make_tmap(&ta, Xp, H, BT, ldx * 2, 64, 128) || !make_tmap(&tb, Wc, H, cols, ldw * 2, 64, eg.b_box_rows) ||
+          !make_out_tmap(&te, E, BT, cols, vc))
+        return FLCE_ERR_CUDA;
+      TcParams prm;
+      std::memset(&prm, 0, sizeof(prm));
+      prm.nprob = 1;
+      TcProblem P = make_problem(eg, (int)BT, cols, (int)H, 0, 0, EPI_DLOGITS, 1);
+      P.group_m = 16;  // a group's X rows (16 x 256 rows) stay in L2 while it sweeps the chunk's columns
+      prm.prob[0] = P;
+      prm.lg.target = tgt;
+      prm.lg.ignore_index = ignore_index;
+      prm.lg.V = V;
+      prm.lg.lse = lse;
+      prm.lg.n_valid = nvalid;
+      prm.lg.reduction = reduction;
+      prm.lg.row_grad = row_grad;
+      prm.lg.v0 = v0;
+      prm.err = dev->err;
+      st = L.run(1, [&] { launch_tc(eg, ta, tb, z, z, prm, dev, stream, &te); });
+      if (st != FLCE_OK) return st;
+    }
+    CUtensorMap tm[4], tc[2];
+    std::memset(tm, 0, sizeof(tm));
+    std::memset(tc, 0, sizeof(tc));
+    TcParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.err = dev->err;
+    int np = 0;
+    if (want_gx) {
+      // grad_X (+)= dz_c W_c: dz K-major [BT, cols], W_c MN-major [cols, H]
+      if (!make_tmap(&tm[2 * np], E, cols, BT, vc * 2, 64, TC_BM) || !make_tmap(&tm[2 * np + 1], Wc, H, cols, ldw * 2, 64, 64))
+        return FLCE_ERR_CUDA;
+      TcProblem P = make_problem(eg, (int)BT, (int)H, cols, 0, 1, EPI_GRADW, 1);
+      P.group_m = 16;
+      P.out = grad_X->data;
+      P.ldo = grad_X->stride[0];
+      P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
+      if (!make_out_tmap(&tc[np], P.out, BT, H, grad_X->stride[0])) return FLCE_ERR_CUDA;
+      prm.prob[np++] = P;
+    }
+    if (want_gw) {
+      // grad_W[v0 : v0 + cols] = dz_c^T X: dz MN-major (K = BT), X MN-major
+      if (!make_tmap(&tm[2 * np], E, cols, BT, vc * 2, 64, 64) || !make_tmap(&tm[2 * np + 1], Xp, H, BT, ldx * 2, 64, 64))
+        return FLCE_ERR_CUDA;
+      TcProblem P = make_problem(eg, cols, (int)H, (int)BT, 1, 1, EPI_GRADW, 0);
+      P.out = static_cast<__nv_bfloat16*>(grad_W->data) + v0 * grad_W->stride[0];
+      P.ldo = grad_W->stride[0];
+      P.gw_mode = GW_STORE_BF16;
+      if (!make_out_tmap(&tc[np], P.out, cols, H, grad_W->stride[0])) return FLCE_ERR_CUDA;
+      prm.prob[np++] = P;
+    }
+    const int64_t units = dev->pairs;
+    if (np == 2 && !grad_combined((int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n, units)) {
+      TcParams p1 = prm, p2 = prm;
+      p1.nprob = 1;
+      p1.prob[1] = TcProblem{};
+      p2.nprob = 1;
+      p2.prob[0] = prm.prob[1];
+      p2.prob[1] = TcProblem{};
+      st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0]); });
+      if (st != FLCE_OK) return st;
+      st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1]); });
+    } else {
+      prm.nprob = np;
+      st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], &tc[1]); });
+    }
+    if (st != FLCE_OK) return st;
+  }
+  return FLCE_OK;
 }
 
 // ------------------------------------------------------------------ FLCE
@@ -505,6 +730,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     for (int k = 0; k < opt->n_shards; ++k)
       if (k * opt->shard_rows < V && (!opt->grad_w_shards[k] || !is_aligned(opt->grad_w_shards[k], 16)))
         return FLCE_ERR_INVALID_ARG;
+    if (!engine().pair) return FLCE_ERR_INVALID_ARG;  // shard routing lives in the pair engine's epilogue
   }
   if (dt == FLCE_BF16) {
     // TMA and 16-byte vector stores: 16-byte aligned bases and rows
@@ -519,6 +745,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   if (keep && from_kept) return FLCE_ERR_INVALID_ARG;
   if ((keep || from_kept) && !opt->workspace) return FLCE_ERR_INVALID_ARG;  // must outlive the call
   if (keep && (grad_X || grad_W || sharded)) return FLCE_ERR_INVALID_ARG;
+  if (opt && (opt->flags & FLCE_FLAG_RECOMPUTE) && !engine().pair) return FLCE_ERR_INVALID_ARG;
   const bool want_gx = grad_X != nullptr && BT > 0;
   const bool want_gw = grad_W != nullptr || sharded;
   const bool need_rowloss = reduction != FLCE_NONE && !(opt && opt->row_loss);
@@ -568,6 +795,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   float* xpart = pl.xpart_elems ? reinterpret_cast<float*>(base + pl.off_xpart) : nullptr;
   float* lse_out = opt ? opt->lse : nullptr;
   float* lse_kept = pl.keep ? reinterpret_cast<float*>(base + pl.off_lse) : nullptr;
+  __nv_bfloat16* gw_local = pl.gw_local ? reinterpret_cast<__nv_bfloat16*>(base + pl.off_gwl) : nullptr;
   const int64_t* tgt = static_cast<const int64_t*>(target->data);
 
   // A0: N (always run: it also flags targets outside [0, V))
@@ -578,7 +806,15 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
 
   const int64_t ldx = X->stride[0], ldw = W->stride[0];
   const Engine eg = engine();
-  for (int64_t c = 0; c < pl.n_chunks; ++c) {
+  if (pl.recompute) {
+    st = run_recompute_passes(X, W, tgt, ignore_index, reduction, grad_X, grad_W, want_gx, want_gw, pl, base,
+                              nvalid, row_loss, row_grad, lse_out, eg, dev, stream, L);
+    if (st != FLCE_OK) return st;
+  }
+  // the stored-chunk schedule (the recompute schedule ran above instead)
+  const int64_t stored_chunks = pl.recompute ? 0 : pl.n_chunks;
+  for (int64_t c = 0; c < stored_chunks; ++c) {
+    L.chunk = c;
     const int64_t r0 = c * pl.chunk;
     const int rows = (int)std::min<int64_t>(pl.chunk, BT - r0);
     const int64_t* tgt_c = tgt + r0;
@@ -604,6 +840,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         prm.nprob = 1;
         prm.prob[0] = make_problem(eg, rows, (int)V, (int)H, 0, 0, EPI_LOGITS, 1);
         prm.lg = LogitsArgs{tgt_c, ignore_index, V, E, pl.lde, pm, ps, pl.ldp, zt};
+        prm.lg.store = 1;
         prm.err = dev->err;
         // the pair engine writes the chunk store through TMA boxes
         CUtensorMap te;
@@ -670,6 +907,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       prm.err = dev->err;
       int np = 0;
       int gx_split = 1;
+      bool gx_wide = false;  // grad_X on 256 x 512 tiles (then launched on its own)
       if (want_gx) {
         if (!make_tmap(&tm[2 * np], E, V, rows, pl.lde * 2, 64, TC_BM) ||
             !make_tmap(&tm[2 * np + 1], Wp, H, V, ldw * 2, 64, 64))
@@ -690,6 +928,10 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
           P.split_stride = (int64_t)rows * H;
           gx_split = P.ksplit;
         }
+        if (eg.pair && gx_split == 1 && gradx_wide(P.tiles_m, H, dev->pairs)) {
+          gx_wide = true;
+          P.tiles_n = (int)ceil_div(H, T2W_BN);
+        }
         prm.prob[np++] = P;
       }
       if (want_gw) {
@@ -697,8 +939,14 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
             !make_tmap(&tm[2 * np + 1], Xc, H, rows, ldx * 2, 64, 64))
           return FLCE_ERR_CUDA;
         TcProblem P = make_problem(eg, (int)V, (int)H, rows, 1, 1, EPI_GRADW, 0);
-        if (sharded) {
-          if (!eg.pair) return FLCE_ERR_INVALID_ARG;  // shard routing lives in the pair engine's epilogue
+        const bool last = c == pl.n_chunks - 1;
+        if (gw_local && !last) {
+          // shards, chunk before the last: accumulate locally (store, then L2 adds)
+          P.out = gw_local;
+          P.ldo = H;
+          if (!make_out_tmap(&tc[np], gw_local, V, H, H)) return FLCE_ERR_CUDA;
+          P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
+        } else if (sharded) {
           P.n_shards = opt->n_shards;
           P.shard_rows = opt->shard_rows;
           P.gw_mode = GW_ADD_BF16;
@@ -709,21 +957,29 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
                                opt->grad_w_shard_ld))
               return FLCE_ERR_CUDA;
           }
+          // the last chunk adds the earlier chunks' local sum to each box on its way to the owner
+          if (gw_local) {
+            P.gw_local = gw_local;
+            P.ld_local = H;
+          }
+          P.gw_mode = GW_ADD_BF16;
         } else {
           P.out = grad_W->data;
           P.ldo = grad_W->stride[0];
           if (!make_out_tmap(&tc[np], P.out, V, H, grad_W->stride[0])) return FLCE_ERR_CUDA;
+          if (!pl.facc) P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
+          else P.gw_mode = c == 0 ? GW_STORE_F32 : (last ? GW_FINAL_F32 : GW_ADD_F32);
         }
-        const bool last = c == pl.n_chunks - 1;
-        if (sharded) P.gw_mode = GW_ADD_BF16;
-        else if (!pl.facc) P.gw_mode = c == 0 ? GW_STORE_BF16 : GW_ADD_BF16;
-        else P.gw_mode = c == 0 ? GW_STORE_F32 : (last ? GW_FINAL_F32 : GW_ADD_F32);
         P.facc = facc;
         P.ld_facc = H;
         prm.prob[np++] = P;
       }
+      // this chunk's grad_W boxes go to the owner shards (the last chunk, or every
+      // chunk when there is no local accumulation)
+      const bool route = sharded && want_gw && (!gw_local || c == pl.n_chunks - 1);
       const int64_t units = eg.pair ? dev->pairs : dev->sms;
-      if (np == 2 && !grad_combined((int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n * prm.prob[0].ksplit, units)) {
+      if (np == 2 && (gx_wide || !grad_combined((int64_t)prm.prob[0].tiles_m * prm.prob[0].tiles_n * prm.prob[0].ksplit,
+                                                 units))) {
         // grad_X and grad_W as two launches: they contend for L2 when interleaved
         TcParams p1 = prm;
         p1.nprob = 1;
@@ -734,14 +990,18 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         p2.prob[1] = TcProblem{};
         CUtensorMap z;
         std::memset(&z, 0, sizeof(z));
-        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0]); });
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0], nullptr, nullptr, gx_wide); });
         if (st != FLCE_OK) return st;
         st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1], nullptr,
-                                      sharded ? &shard_maps : nullptr); });
+                                      route ? &shard_maps : nullptr); });
+      } else if (np == 1 && gx_wide) {
+        prm.nprob = 1;
+        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], nullptr, nullptr,
+                                      true); });
       } else {
         prm.nprob = np;
         st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], &tc[1],
-                                      sharded ? &shard_maps : nullptr); });
+                                      route ? &shard_maps : nullptr); });
       }
       if (st != FLCE_OK) return st;
       if (gx_split > 1) {
@@ -786,6 +1046,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
       }
     }
   }
+  L.chunk = -1;
   if (reduction != FLCE_NONE && !from_kept) {
     st = L.run(5, [&] {
       finalize_loss_kernel<<<1, 1024, 0, stream>>>(row_loss, BT, nvalid, reduction,
@@ -1071,6 +1332,39 @@ flce_status run_ce_noalloc(const flce_tensor* Z, const flce_tensor* target, int6
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
+// The engine on a plain GEMM (flce_gemm_bf16), optionally with the failure-path
+// test hook (test_stall = output tile number + 1, 0 = off).
+flce_status run_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K, int64_t lda,
+                          int64_t ldb, int64_t ldc, int32_t a_mn_major, int32_t b_mn_major, int test_stall,
+                          cudaStream_t stream) {
+  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0) return FLCE_ERR_INVALID_ARG;
+  if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return FLCE_ERR_INVALID_ARG;
+  if (lda % 8 || ldb % 8 || ldc % 4) return FLCE_ERR_INVALID_ARG;
+  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16)) return FLCE_ERR_INVALID_ARG;
+  if (lda < (a_mn_major ? M : K) || ldb < (b_mn_major ? N : K) || ldc < N) return FLCE_ERR_INVALID_ARG;
+  DeviceCtx* dev = nullptr;
+  const flce_status st = device_ctx(&dev);
+  if (st != FLCE_OK) return st;
+  CUtensorMap ta, tb, z;
+  std::memset(&z, 0, sizeof(z));
+  const Engine eg = engine();
+  const bool ok = (a_mn_major ? make_tmap(&ta, A, M, K, lda * 2, 64, 64) : make_tmap(&ta, A, K, M, lda * 2, 64, 128)) &&
+                  (b_mn_major ? make_tmap(&tb, B, N, K, ldb * 2, 64, 64) : make_tmap(&tb, B, K, N, ldb * 2, 64, eg.b_box_rows));
+  if (!ok) return FLCE_ERR_CUDA;
+  TcParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.nprob = 1;
+  prm.prob[0] = make_problem(eg, (int)M, (int)N, (int)K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, EPI_STORE_F32, 1);
+  prm.prob[0].out = C;
+  prm.prob[0].ldo = ldc;
+  prm.err = dev->err;
+  prm.test_stall = test_stall;
+  launch_tc(eg, ta, tb, z, z, prm, dev, stream);
+  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
+  if (env_debug() && cudaStreamSynchronize(stream) != cudaSuccess) return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
+
 }  // namespace
 }  // namespace flce
 
@@ -1087,6 +1381,7 @@ flce_status flce_fwd_bwd_ex(const flce_tensor* X, const flce_tensor* W, const fl
                             flce_tensor* grad_X, flce_tensor* grad_W, flce_stream_t stream,
                             const flce_options* opt, flce_stats* stats) {
   try {
+    const NvtxRange range("flce_fwd_bwd");
     return run_flce(X, W, target, ignore_index, reduction, loss, grad_X, grad_W,
                     reinterpret_cast<cudaStream_t>(stream), opt, stats);
   } catch (...) {
@@ -1141,6 +1436,7 @@ flce_status flce_cross_entropy(const flce_tensor* logits, const flce_tensor* tar
                                flce_tensor* grad_logits, flce_stream_t stream,
                                const flce_options* opt) {
   try {
+    const NvtxRange range("flce_cross_entropy");
     return run_ce(logits, target, ignore_index, reduction, loss, grad_logits,
                   reinterpret_cast<cudaStream_t>(stream), opt);
   } catch (...) {
@@ -1162,32 +1458,16 @@ flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const flce_ten
 flce_status flce_gemm_bf16(const void* A, const void* B, float* C, int64_t M, int64_t N,
                            int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t a_mn_major,
                            int32_t b_mn_major, flce_stream_t stream) {
-  if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0) return FLCE_ERR_INVALID_ARG;
-  if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return FLCE_ERR_INVALID_ARG;
-  if (lda % 8 || ldb % 8 || ldc % 4) return FLCE_ERR_INVALID_ARG;
-  if (!is_aligned(A, 16) || !is_aligned(B, 16) || !is_aligned(C, 16)) return FLCE_ERR_INVALID_ARG;
-  if (lda < (a_mn_major ? M : K) || ldb < (b_mn_major ? N : K) || ldc < N) return FLCE_ERR_INVALID_ARG;
-  DeviceCtx* dev = nullptr;
-  const flce_status st = device_ctx(&dev);
-  if (st != FLCE_OK) return st;
-  CUtensorMap ta, tb, z;
-  std::memset(&z, 0, sizeof(z));
-  const Engine eg = engine();
-  const bool ok = (a_mn_major ? make_tmap(&ta, A, M, K, lda * 2, 64, 64) : make_tmap(&ta, A, K, M, lda * 2, 64, 128)) &&
-                  (b_mn_major ? make_tmap(&tb, B, N, K, ldb * 2, 64, 64) : make_tmap(&tb, B, K, N, ldb * 2, 64, eg.b_box_rows));
-  if (!ok) return FLCE_ERR_CUDA;
-  TcParams prm;
-  std::memset(&prm, 0, sizeof(prm));
-  prm.nprob = 1;
-  prm.prob[0] = make_problem(eg, (int)M, (int)N, (int)K, a_mn_major ? 1 : 0, b_mn_major ? 1 : 0, EPI_STORE_F32, 1);
-  prm.prob[0].out = C;
-  prm.prob[0].ldo = ldc;
-  prm.err = dev->err;
-  launch_tc(eg, ta, tb, z, z, prm, dev, reinterpret_cast<cudaStream_t>(stream));
-  if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
-  if (env_debug() && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return FLCE_ERR_CUDA;
-  return FLCE_OK;
+  return run_gemm_bf16(A, B, C, M, N, K, lda, ldb, ldc, a_mn_major, b_mn_major, 0,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_gemm_bf16_wait_test(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
+                                     int64_t lda, int64_t ldb, int64_t ldc, int32_t stall_tile,
+                                     flce_stream_t stream) {
+  if (stall_tile < 0) return FLCE_ERR_INVALID_ARG;
+  if (!engine().pair) return FLCE_ERR_INVALID_ARG;  // the hook lives in the pair engine
+  return run_gemm_bf16(A, B, C, M, N, K, lda, ldb, ldc, 0, 0, stall_tile + 1, reinterpret_cast<cudaStream_t>(stream));
 }
 
 flce_status flce_scale_grad(flce_tensor* t, const float* scale, flce_stream_t stream) {

@@ -45,6 +45,7 @@ enum EpiKind : int {
   EPI_STORE_BF16 = 1,
   EPI_GRADW = 2,
   EPI_STORE_F32 = 3,
+  EPI_DLOGITS = 4,  // recompute schedule: dz = (exp(z - lse) - onehot) * scale, stored bf16
 };
 
 enum GradWMode : int {
@@ -68,6 +69,10 @@ struct TcProblem {
   int64_t ld_facc;
   int n_shards;        // EPI_GRADW: > 0 routes each output box to its owner shard (add)
   int64_t shard_rows;  // rows per shard (multiple of 32)
+  const void* gw_local;  // EPI_GRADW with shards: bf16 [M, ld_local] partial sum of the earlier
+  int64_t ld_local;      // chunks, added to this tile before it goes to the owner shard (or null)
+  int group_m;         // > 0: tiles run in groups of group_m tile rows, m fastest inside a group
+                       // (each B column tile is reused by the group's rows while they share L2)
   int ksplit;          // split-K factor (>= 1): tile t covers K-blocks of split t / (tiles_m*tiles_n)
   int kb_per_split;    // K-blocks per split
   int64_t split_stride;  // elements between the output slices of consecutive splits
@@ -88,6 +93,14 @@ struct LogitsArgs {
   float* part_s;           // [ntile, ldp]: per (tile, row) sum of exp(z - m_tile)
   int64_t ldp;
   float* zt;               // [rows]: z at the target column
+  int store;               // EPI_LOGITS on the pair engine: 0 = partials only, no store
+  // EPI_DLOGITS (recompute schedule): columns [0, N) of the launch are vocabulary
+  // columns [v0, v0 + N); V above is the whole vocabulary (for target validity)
+  const float* lse;        // [rows]: row logsumexp from the first pass
+  const int64_t* n_valid;  // mean denominator N (device)
+  int reduction;           // 0 mean (scale 1/N), 1 sum, 2 none
+  const float* row_grad;   // [rows] upstream gradient per row, or null (all ones)
+  int64_t v0;
 };
 
 struct TcParams {
@@ -95,6 +108,10 @@ struct TcParams {
   int nprob;
   LogitsArgs lg;
   uint32_t* err;
+  // Test of the failure path (pair engine; 0 = off): the MMA issuer waits, before
+  // its output tile number test_stall - 1, on a barrier nothing arrives on, so the
+  // bounded wait runs out and the kernel takes its abort path.
+  int test_stall;
 };
 
 // ------------------------------------------------------------ tile schedule
@@ -156,7 +173,15 @@ __device__ __forceinline__ Tile sched_tile(const TcParams& p, const TileSched& s
   const int per_split = P.tiles_m * P.tiles_n;
   T.split = t / per_split;
   t -= T.split * per_split;
-  if (P.m_fastest) {
+  if (P.group_m > 0) {
+    const int per_group = P.group_m * P.tiles_n;
+    const int grp = t / per_group;
+    const int first_m = grp * P.group_m;
+    const int gm = min(P.group_m, P.tiles_m - first_m);
+    const int w = t - grp * per_group;
+    T.tm = first_m + w % gm;
+    T.tn = w / gm;
+  } else if (P.m_fastest) {
     T.tm = t % P.tiles_m;
     T.tn = t / P.tiles_m;
   } else {

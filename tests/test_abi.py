@@ -312,3 +312,90 @@ def test_chunk_rows_environment_override(lib, monkeypatch):
     for bad in ("", "abc", "-5", "0", "12x"):
         monkeypatch.setenv("FLCE_CHUNK_ROWS", bad)
         assert plan() == default, bad
+
+
+def _nvtx_recorder(tmp_path):
+    """Build tests/c/nvtx_record.c, a minimal NVTX tool that logs range pushes and pops."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    so = tmp_path / "nvtx_record.so"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-shared", "-fPIC", "-I", "/usr/local/cuda/include",
+                        os.path.join(ROOT, "tests", "c", "nvtx_record.c"), "-o", str(so)],
+                       capture_output=True, text=True)
+    if r.returncode != 0 and "nvToolsExt.h" in r.stderr:
+        pytest.skip("NVTX 3 headers not found")
+    assert r.returncode == 0, r.stderr
+    return so
+
+
+def run_with_nvtx(tmp_path, code):
+    """Run `code` in a fresh Python with the NVTX recorder injected; return the logged lines."""
+    import subprocess
+    import sys
+
+    so = _nvtx_recorder(tmp_path)
+    log = tmp_path / "nvtx.log"
+    env = dict(os.environ, NVTX_INJECTION64_PATH=str(so), FLCE_NVTX_LOG=str(log), PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    return log.read_text().splitlines() if log.exists() else []
+
+
+def test_nvtx_range_around_each_call(tmp_path, lib):
+    """Every compute entry point opens an NVTX range for its call, closed on
+    every return path (here: an argument error, found before any device work)."""
+    code = ("from linear_cross_entropy_04_b200 import _binding as B\n"
+            "L = B.lib()\n"
+            "assert L.flce_fwd_bwd(None, None, None, -100, 0, None, None, None, None) == 1\n"
+            "assert L.flce_cross_entropy(None, None, -100, 0, None, None, None, None) == 1\n")
+    assert run_with_nvtx(tmp_path, code) == ["push flce_fwd_bwd", "pop", "push flce_cross_entropy", "pop"]
+
+
+def test_recompute_schedule_plan(lib):
+    """The recompute schedule's workspace: the [BT, Vc] store with Vc from the
+    option or the budget, plus per-row lse / losses and one row block's partials;
+    it refuses f32, the two-phase flags and grad_W shards on the host."""
+    from linear_cross_entropy_04_b200.api import plan
+
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    BT, H, V = 4096, 4096, 128256
+    p = plan(BT, H, V, schedule="recompute", chunk_rows=1000)
+    assert p["chunk_rows"] == 1024 and p["n_chunks"] == -(-V // 1024)
+    ntile = -(-V // 256)
+    expect = a256(8) + a256(4 * BT) + a256(4 * 4096) + 2 * a256(4 * ntile * 4096) + a256(BT * 1024 * 2) + a256(4 * BT)
+    assert p["workspace_bytes"] == expect
+    q = plan(BT, H, V, schedule="recompute", workspace_limit_bytes=64 << 20)
+    assert q["chunk_rows"] == (64 << 20) // (BT * 2) // 256 * 256 == 8192
+    d = plan(BT, H, V, schedule="recompute")
+    assert d["chunk_rows"] == 65536 and d["n_chunks"] == 2   # 512 MiB over 4096 rows
+    tiny = plan(BT, H, V, schedule="recompute", chunk_rows=1)
+    assert tiny["chunk_rows"] == 256 and tiny["workspace_bytes"] < plan(BT, H, V)["workspace_bytes"] / 8
+    whole = plan(100, 64, 1000, schedule="recompute", chunk_rows=5000)
+    assert whole["chunk_rows"] == 1024 and whole["n_chunks"] == 1  # capped at V rounded up to 256
+    st = B.FlceStats()
+    for flags, dt, code in ((B.FLAG_RECOMPUTE, B.F32, 2), (B.FLAG_RECOMPUTE | B.FLAG_KEEP_LOGITS, B.BF16, 1),
+                            (B.FLAG_RECOMPUTE | B.FLAG_FROM_KEPT, B.BF16, 1)):
+        o = B.FlceOptions()
+        lib.flce_options_init(ctypes.byref(o))
+        o.flags = flags
+        assert lib.flce_plan(BT, H, V, dt, 1, ctypes.byref(o), ctypes.byref(st)) == code, (flags, dt)
+    o = B.FlceOptions()
+    lib.flce_options_init(ctypes.byref(o))
+    o.flags = B.FLAG_RECOMPUTE
+    o.n_shards, o.shard_rows = 2, 64128
+    assert lib.flce_plan(BT, H, V, B.BF16, 1, ctypes.byref(o), ctypes.byref(st)) == 1
+    with pytest.raises(ValueError, match="schedule"):
+        plan(BT, H, V, schedule="vocab")
+
+
+def test_wait_test_hook_validates(lib, monkeypatch):
+    """flce_gemm_bf16_wait_test refuses, on the host, what flce_gemm_bf16 refuses, a
+    negative stall tile, and the single-CTA engine (the hook lives in the pair engine)."""
+    assert lib.flce_gemm_bf16_wait_test(None, None, None, 1, 1, 1, 8, 8, 4, 0, None) == 1
+    assert lib.flce_gemm_bf16_wait_test(FAKE, FAKE, FAKE, 16, 16, 16, 16, 16, 16, -1, None) == 1
+    monkeypatch.setenv("FLCE_ENGINE", "1sm")
+    assert lib.flce_gemm_bf16_wait_test(FAKE, FAKE, FAKE, 256, 256, 64, 64, 64, 256, 0, None) == 1

@@ -5,7 +5,8 @@ error <= 1e-3; grad_X, grad_W: max |gpu - ref| <= 2e-2 * max |ref|):
 
   * the bench workload (Llama-3-8B lm_head, 4096 x 4096 x 128256) whole: the
     loss, every per-row loss and every element of grad_X and grad_W against
-    the float64 oracle over the whole batch;
+    the float64 oracle over the whole batch, on the stored-chunk schedule and
+    on the recompute schedule (2 and 16 vocabulary chunks);
   * the four large workloads at full size with W = 0, in both grad_W
     accumulation modes: loss = ln V, grad_X = 0 exactly, and every element of
     grad_W against its closed form ((1/V) sum_valid X_i - sum_{valid, t_i = v}
@@ -73,6 +74,18 @@ def test_bench_workload_whole_batch_against_the_oracle():
     np.testing.assert_allclose(row_loss.cpu().numpy(), ref["row_loss"], rtol=1e-3, atol=1e-3)
     assert_close_blockwise(gX, ref["grad_X"], "grad_X")
     assert_close_blockwise(gW, ref["grad_W"], "grad_W")
+    # the recompute schedule on the same batch: its default (2 vocabulary chunks of
+    # 65536 columns) and a 64 MiB store (16 chunks of 8192)
+    for budget, n in ((0, 2), (64 << 20, 16)):
+        loss, gX, gW, st = L().fused_linear_cross_entropy(X, W, t, row_loss=row_loss, schedule="recompute",
+                                                           workspace_limit_bytes=budget, return_stats=True)
+        torch.cuda.synchronize()
+        assert L().device_error() == 0
+        assert st["n_chunks"] == n
+        assert rel_err(loss.item(), ref["loss"]) <= 1e-3, (loss.item(), ref["loss"])
+        np.testing.assert_allclose(row_loss.cpu().numpy(), ref["row_loss"], rtol=1e-3, atol=1e-3)
+        assert_close_blockwise(gX, ref["grad_X"], f"grad_X (recompute, {n} chunks)")
+        assert_close_blockwise(gW, ref["grad_W"], f"grad_W (recompute, {n} chunks)")
 
 
 _x_cache = {}

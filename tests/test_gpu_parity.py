@@ -23,13 +23,13 @@ def L():
 
 
 def run_case(d, reduction="mean", chunk_rows=0, grad_w_accum="output", ignore_index=IGNORE_INDEX,
-             want_grad_X=True, want_grad_W=True):
+             want_grad_X=True, want_grad_W=True, **kw):
     X, W, t = to_dev(d)
     row_loss = torch.empty(d["BT"], dtype=torch.float32, device="cuda")
     loss, gX, gW, st = L().fused_linear_cross_entropy(
         X, W, t, ignore_index=ignore_index, reduction=reduction, chunk_rows=chunk_rows,
         grad_w_accum=grad_w_accum, row_loss=row_loss, want_grad_X=want_grad_X, want_grad_W=want_grad_W,
-        return_stats=True)
+        return_stats=True, **kw)
     torch.cuda.synchronize()
     assert L().device_error() == 0
     ref = oracle.flce(d["X"], d["W"], d["target"], ignore_index=ignore_index, reduction=reduction)
@@ -327,20 +327,33 @@ def test_host_pipeline_matches_device_call():
         assert torch.equal(o[1], ref[1].cpu()) and torch.equal(o[2], ref[2].cpu())
 
 
-@pytest.mark.parametrize("n_shards,shard_rows", [(3, 1024), (4, 800)])
-def test_grad_W_shard_routing(n_shards, shard_rows):
+@pytest.mark.parametrize("every_chunk", [False, True])
+@pytest.mark.parametrize("n_shards,shard_rows,BT,chunk", [(3, 1024, 700, 256), (4, 800, 700, 256),
+                                                         (4, 768, 1100, 128)])
+def test_grad_W_shard_routing(n_shards, shard_rows, BT, chunk, every_chunk):
     """grad_W added tile by tile into shards (the data-parallel reduce-scatter path), with every
-    shard on this GPU: shard k must hold rows [k*shard_rows, ...) of the plain grad_W."""
-    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=700, H=256, V=3000)
+    shard on this GPU: shard k must hold rows [k*shard_rows, ...) of the plain grad_W, bit for
+    bit, whether the chunks before the last accumulate locally (the default) or every chunk's
+    boxes are routed (FLAG_ROUTE_EVERY_CHUNK); and match the oracle. The last case runs
+    9 chunks into 4 shards."""
+    from linear_cross_entropy_04_b200 import _binding as B
+
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=BT, H=256, V=3000)
     X, W, t = to_dev(d)
-    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=chunk)
     shards = [torch.zeros(shard_rows, 256, dtype=torch.bfloat16, device="cuda") for _ in range(n_shards)]
-    loss2, gX2, gW2 = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256, grad_w_shards=shards,
-                                                     shard_rows=shard_rows)
+    flags = B.FLAG_ROUTE_EVERY_CHUNK if every_chunk else 0
+    loss2, gX2, gW2, st = L().fused_linear_cross_entropy(X, W, t, chunk_rows=chunk, grad_w_shards=shards,
+                                                         shard_rows=shard_rows, flags=flags, return_stats=True)
     torch.cuda.synchronize()
+    assert L().device_error() == 0
+    assert st["n_chunks"] == -(-BT // chunk)
+    plain = L().plan(BT, 256, 3000, chunk_rows=chunk)["workspace_bytes"]
+    local = 0 if every_chunk else 3000 * 256 * 2  # the earlier chunks' local bf16 sum
+    assert st["workspace_bytes"] - plain == local
     assert gW2 is None and loss2.item() == loss.item() and torch.equal(gX2, gX)
     joined = torch.cat(shards)[:3000]
-    assert torch.equal(joined, gW)  # same adds, same order
+    assert torch.equal(joined, gW)  # same roundings in the same order
     assert torch.all(torch.cat(shards)[3000:] == 0)
     ref = oracle.flce(d["X"], d["W"], d["target"])
     assert_grad_close(joined, ref["grad_W"], "bf16", "sharded grad_W")
@@ -517,6 +530,28 @@ def test_engine_variants_match_oracle(monkeypatch, env):
     assert_grad_close(gW, ref["grad_W"], "bf16", f"grad_W {env}")
 
 
+# grad_X on the pair engine's 256 x 512 tiles, forced on and off: a ragged last
+# 512-column tile (H = 264, 776: the second half of the last tile lies partly or
+# wholly outside), several waves of wide tiles on 74 pairs (BT = 4200 in one
+# chunk, H = 2560: 17 x 5 tiles), and chunk rows that are not a tile multiple.
+@pytest.mark.parametrize("tile", ["wide", "narrow"])
+@pytest.mark.parametrize("BT,H,V,chunk", [(500, 264, 3000, 384), (300, 776, 2000, 0), (4200, 2560, 1000, 4224),
+                                          (700, 512, 9000, 256)])
+def test_gradx_tile_width_matches_oracle(monkeypatch, tile, BT, H, V, chunk):
+    monkeypatch.setenv("FLCE_GRADX_TILE", tile)
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=BT, H=H, V=V)
+    X, W, t = to_dev(d)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=chunk)
+    gX_only = L().fused_linear_cross_entropy(X, W, t, chunk_rows=chunk, want_grad_W=False)[1]
+    torch.cuda.synchronize()
+    assert L().device_error() == 0
+    assert torch.equal(gX, gX_only)
+    ref = oracle.flce(d["X"], d["W"], d["target"])
+    assert rel_err(loss.item(), ref["loss"]) <= TOL["bf16"]["loss"]
+    assert_grad_close(gX, ref["grad_X"], "bf16", f"grad_X ({tile})")
+    assert_grad_close(gW, ref["grad_W"], "bf16", f"grad_W ({tile})")
+
+
 # Degenerate shapes of the method: a one-class vocabulary (every row's loss and
 # gradient are exactly 0), two classes (the logistic loss), a single row, and
 # the smallest hidden size with an odd vocabulary.
@@ -544,3 +579,87 @@ def test_one_class_vocabulary_is_exactly_zero(wl):
     lz, dz = L().cross_entropy(z, torch.zeros(7, dtype=torch.int64, device="cuda"))
     torch.cuda.synchronize()
     assert abs(lz.item()) <= 1e-6 and dz.float().abs().max().item() <= 1e-6
+
+
+def test_nvtx_ranges_per_phase_and_chunk(tmp_path):
+    """With an NVTX tool attached, a call shows as one range holding a range per
+    phase launch, named with its row chunk, in launch order."""
+    from test_abi import run_with_nvtx
+
+    code = ("import torch\n"
+            "import linear_cross_entropy_04_b200 as flce\n"
+            "X = torch.randn(700, 256, device='cuda').to(torch.bfloat16)\n"
+            "W = (torch.randn(3000, 256, device='cuda') * 0.02).to(torch.bfloat16)\n"
+            "t = torch.randint(0, 3000, (700,), device='cuda')\n"
+            "flce.fused_linear_cross_entropy(X, W, t, chunk_rows=256)\n"
+            "torch.cuda.synchronize()\n")
+    lines = run_with_nvtx(tmp_path, code)
+    depth = 0
+    for ln in lines:
+        depth += 1 if ln.startswith("push") else -1
+        assert depth >= 0
+    assert depth == 0
+    pushes = [ln[5:] for ln in lines if ln.startswith("push")]
+    assert pushes[0] == "flce_fwd_bwd"
+    assert pushes[1] == "flce count_valid" and pushes[-1] == "flce loss_reduce"
+    body = [p for p in pushes[2:-1]]
+    expect = []
+    for c in range(3):
+        expect += [f"flce logits_gemm_softmax chunk {c}", f"flce row_combine chunk {c}",
+                   f"flce dlogits_inplace chunk {c}"]
+        grads = [p for p in body if p == f"flce grad_gemms chunk {c}"]
+        assert 1 <= len(grads) <= 2
+        expect += grads
+    assert body == expect
+
+
+# ------------------------------------------------------------ recompute schedule
+@pytest.mark.parametrize("BT,H,V,vc", [(700, 256, 3000, 512), (129, 192, 4099, 256), (1000, 512, 3000, 0),
+                                       (300, 8, 1000, 256), (513, 264, 9000, 2048)])
+def test_recompute_schedule_matches_oracle(BT, H, V, vc):
+    """The vocabulary-outer schedule against the oracle: several vocabulary chunks
+    with ragged last chunks, row tails, H = 8, and the default chunk from the budget."""
+    st = run_case(make_inputs(WORKLOADS["llama3_8b_seq"], BT=BT, H=H, V=V), chunk_rows=vc, schedule="recompute")
+    expect_vc = min(-(-V // 256) * 256, -(-vc // 256) * 256) if vc else -(-V // 256) * 256
+    assert st["chunk_rows"] == expect_vc and st["n_chunks"] == -(-V // expect_vc)
+
+
+@pytest.mark.parametrize("reduction", ["sum", "none"])
+def test_recompute_schedule_reductions_and_row_grad(reduction):
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=600, H=128, V=2000)
+    X, W, t = to_dev(d)
+    g = np.random.default_rng(4).standard_normal(600).astype(np.float32)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, reduction=reduction, row_grad=torch.from_numpy(g).cuda(),
+                                                  chunk_rows=512, schedule="recompute")
+    torch.cuda.synchronize()
+    assert L().device_error() == 0
+    ref = oracle.flce(d["X"], d["W"], d["target"], reduction=reduction, row_grad=g)
+    if reduction == "none":
+        np.testing.assert_allclose(loss.cpu().numpy(), ref["loss"], rtol=1e-3, atol=1e-3)
+    else:
+        assert rel_err(loss.item(), ref["loss"]) <= 1e-3
+    assert_grad_close(gX, ref["grad_X"], "bf16", "grad_X (recompute)")
+    assert_grad_close(gW, ref["grad_W"], "bf16", "grad_W (recompute)")
+
+
+def test_recompute_schedule_edge_cases():
+    """ignore_index inside the vocabulary, one gradient only, every row ignored,
+    and W = 0 (loss ln V, grad_X exactly 0), on the recompute schedule."""
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=300, H=64, V=1500)
+    d["target"][::7] = 5
+    run_case(d, ignore_index=5, chunk_rows=256, schedule="recompute")
+    run_case(d, want_grad_X=False, chunk_rows=256, schedule="recompute")
+    run_case(d, want_grad_W=False, chunk_rows=256, schedule="recompute")
+    d2 = make_inputs(WORKLOADS["llama3_8b_seq"], BT=200, H=64, V=1000)
+    d2["target"][:] = IGNORE_INDEX
+    X, W, t = to_dev(d2)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=256, schedule="recompute")
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0 and torch.all(gX == 0) and torch.all(gW == 0)
+    d3 = make_inputs(WORKLOADS["llama3_8b_seq"], BT=500, H=256, V=3000, w_zero=True)
+    X, W, t = to_dev(d3)
+    loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, chunk_rows=1024, schedule="recompute")
+    torch.cuda.synchronize()
+    assert rel_err(loss.item(), np.log(3000)) <= 1e-3
+    assert torch.all(gX == 0)
+    assert_grad_close(gW, oracle.flce(d3["X"], d3["W"], d3["target"])["grad_W"], "bf16", "grad_W (W=0, recompute)")
