@@ -131,6 +131,17 @@ flce_status device_ctx(DeviceCtx** out) {
           c.ce_max_cluster = CER_MAX_CLUSTER;
       }
       cudaGetLastError();
+      // Load the upstream-gradient kernels now: under lazy module loading a
+      // kernel's first launch can block the host, and these run inside autograd's
+      // backward, which must not wait for the GPU.
+      {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, scale_grad_kernel<__nv_bfloat16, 8>) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, scale_grad_kernel<__nv_bfloat16, 1>) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, scale_grad_kernel<float, 4>) != cudaSuccess ||
+            cudaFuncGetAttributes(&fa, scale_grad_kernel<float, 1>) != cudaSuccess)
+          return FLCE_ERR_CUDA;
+      }
       // A private pool that keeps freed workspace mapped, so repeated calls
       // reuse it stream-ordered instead of mapping and unmapping memory.
       cudaMemPoolProps pp;
