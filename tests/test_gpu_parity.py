@@ -646,8 +646,10 @@ def test_recompute_schedule_edge_cases():
     """ignore_index inside the vocabulary, one gradient only, every row ignored,
     and W = 0 (loss ln V, grad_X exactly 0), on the recompute schedule."""
     d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=300, H=64, V=1500)
+    d["target"][d["target"] == IGNORE_INDEX] = 5  # -100 would be an out-of-range target with ignore_index 5
     d["target"][::7] = 5
     run_case(d, ignore_index=5, chunk_rows=256, schedule="recompute")
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=300, H=64, V=1500)
     run_case(d, want_grad_X=False, chunk_rows=256, schedule="recompute")
     run_case(d, want_grad_W=False, chunk_rows=256, schedule="recompute")
     d2 = make_inputs(WORKLOADS["llama3_8b_seq"], BT=200, H=64, V=1000)
