@@ -625,6 +625,9 @@ def main():
             "peak_kind": f"{peaks['source']} burst bf16 (timed region {ms / 1e3:.2f} s)",
             "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
             "launches": gemm_launches, "avg_launch_ms": gemm_ms / max(gemm_launches, 1),
+            # HBM GB/s of the GEMM launches: the recorded per-launch DRAM bytes over this run's launch time
+            "hbm_gbs": (traffic["bytes_per_launch"] / (gemm_ms / max(gemm_launches, 1) / 1e3) / 1e9
+                        if traffic else None),
             # the recompute schedule executes 8*BT*H*V tensor FLOPs for the 6 that count
             "executed_tflops": achieved * (8.0 if args.schedule == "recompute" else 6.0) / 6.0}
     all_ms = sum(v[0] for v in phases.values())

@@ -68,3 +68,33 @@ def test_reference_arm_runs_on_the_host_and_samples_at_most_the_batch():
     assert line["config"]["sample_tokens_per_step"] <= 512
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["value"] > 0 and line["unit"] == "tokens/s"
+
+
+def test_recorded_traffic_follows_the_source_hash(bench, tmp_path, monkeypatch):
+    """The roofline's traffic figure is read from the committed capture only while
+    the five sources that decide the captured launches hash to the recorded value."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    src = tmp_path / "linear_cross_entropy_04_b200" / "csrc"
+    src.mkdir(parents=True)
+    for f in bench.KERNEL_SOURCES:
+        (tmp_path / f).write_text("kernel " + f)
+    assert {os.path.basename(f) for f in bench.KERNEL_SOURCES} >= {"flce.cu", "aux_kernels.cuh", "tc_gemm2.cuh"}
+    h = bench.kernel_source_hash()
+    (prof / "tc_gemm_pair_kernel_toy_dram.md").write_text(
+        f"# toy\n- kernel_source_sha256_16: `{h}`\n- dram_bytes_per_launch: `123456`\n")
+    assert bench.recorded_traffic("toy")["bytes_per_launch"] == 123456.0
+    (tmp_path / bench.KERNEL_SOURCES[-1]).write_text("changed")
+    assert bench.recorded_traffic("toy") is None
+    assert bench.recorded_traffic("no_such_workload") is None
+
+
+def test_workload_size_overrides_rename_the_workload(bench, monkeypatch):
+    import sys
+
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--BT", "1024", "--V", "32768"])
+    w = bench.workload(bench.parse())
+    assert (w.BT, w.H, w.V) == (1024, 4096, 32768) and w.name != "llama3_8b_seq"
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    assert bench.workload(bench.parse()).name == "llama3_8b_seq"
