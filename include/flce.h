@@ -269,9 +269,9 @@ FLCE_API flce_status flce_cross_entropy(const flce_tensor* logits, const flce_te
  *   8 * ceil(V / 1024) + 12 bytes per row (round BT up to a multiple of 32
  *   for the first term), e.g. up to ~8200 rows at V = 128256; larger problems
  *   return FLCE_ERR_WORKSPACE_TOO_SMALL before any GPU work.
- *   The first call on a device looks up the array's device address (a CUDA
- *   runtime query, no allocation); make that first call before any stream
- *   capture. All calls share the array and it keeps the last call's contents;
+ *   The first call on a device looks up the array's device address and loads
+ *   every kernel the entry point launches (CUDA runtime queries, no allocation);
+ *   make that first call before any stream capture. All calls share the array and it keeps the last call's contents;
  *   every value a call reads from it is written earlier in the same call.
  *   Calls that overlap on the GPU (on different streams, or from different
  *   threads without ordering) race on the array: order them.

@@ -1232,8 +1232,9 @@ std::mutex g_noalloc_mu;
 NoAllocDevice g_noalloc_dev[kMaxDevices];
 
 // Once per device, with that device current: look up the device addresses of
-// the scratch array and the error word. (In host code the array's name is only
-// a host-side stand-in; the kernels must be given the address found here.)
+// the scratch array and the error word, and load the kernels the entry point
+// launches. (In host code the array's name is only a host-side stand-in; the
+// kernels must be given the address found here.)
 flce_status noalloc_device(NoAllocDevice** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
@@ -1250,6 +1251,17 @@ flce_status noalloc_device(NoAllocDevice** out) {
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.scratch), g_noalloc_scratch) != cudaSuccess)
         return FLCE_ERR_CUDA;
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_err_word) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+      // load every kernel this entry point launches, so that no later call is the
+      // first launch of one of them (under lazy module loading that may block the host)
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, count_valid_kernel) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, ce_partials_kernel<__nv_bfloat16>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, ce_partials_kernel<float>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, combine_kernel) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, ce_grad_kernel<__nv_bfloat16>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, ce_grad_kernel<float>) != cudaSuccess ||
+          cudaFuncGetAttributes(&fa, finalize_loss_kernel) != cudaSuccess)
         return FLCE_ERR_CUDA;
     }
     d.init = true;
