@@ -560,6 +560,157 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
   }
 }
 
+// ------------------------------------------------------------------ one pass, staged in shared memory
+// The same one-pass cross-entropy as ce_row_cluster_kernel (a cluster of C CTAs
+// per row, each reducing its slice, the C (max, sum) pairs exchanged through
+// distributed shared memory), with the slice staged in shared memory instead of
+// registers: one thread moves it in with a single bulk copy (cp.async.bulk,
+// completing on an mbarrier) and the gradient goes back out with another,
+// written in place over the staged logits. The slice (<= 16384 bf16, 32 KB)
+// leaves the registers free, so 6 CTAs share an SM instead of 4, and the
+// copies are issued by the bulk-copy engine rather than 256 threads' loads.
+// Columns past the last 16-byte vector of a slice (V not a multiple of 8)
+// move with plain loads and stores.
+__device__ __forceinline__ void bulk_load_smem(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_store_global(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(smem_src)),
+               "r"(bytes)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, uint32_t* err) {
+  extern __shared__ __align__(128) uint4 zs4[];  // the slice: (slice / 8) 16-byte vectors
+  __shared__ float red[CER_THREADS / 32];
+  __shared__ float2 parts[CER_MAX_CLUSTER];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int no_abort;
+  const uint32_t rank = cluster_ctarank(), csize = cluster_nctarank();
+  const int r = blockIdx.y;
+  const int base = (int)rank * a.slice;
+  const int end = base + a.slice < (int)a.V ? base + a.slice : (int)a.V;
+  const int n = end - base;             // columns of this CTA (>= 1)
+  const int nvec = n >> 3;              // whole 16-byte vectors
+  const int tail = n - (nvec << 3);     // columns after them (< 8)
+  const int nv_all = nvec + (tail ? 1 : 0);
+  const __nv_bfloat16* zr = a.z + (int64_t)r * a.ldz;
+  const int64_t t64 = a.target[r];
+  const bool valid = target_valid(t64, a.V, a.ignore_index);
+  const int t = valid ? (int)t64 : -1;
+  const bool owns_t = valid && t >= base && t < end;
+  if (!valid && !a.lse_out) {
+    // an ignored row needs neither its logits nor a cluster exchange (every CTA of
+    // the cluster takes this branch: they share the row)
+    if (threadIdx.x == 0 && rank == 0) a.row_loss[r] = 0.f;
+    if (a.dz) {
+      __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
+      for (int c = base + (int)threadIdx.x * 8; c < end; c += CER_THREADS * 8) {
+        if (c + 8 <= end) {
+          *reinterpret_cast<uint4*>(dr + c) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          for (int k = c; k < end; ++k) dr[k] = __float2bfloat16_rn(0.f);
+        }
+      }
+    }
+    return;
+  }
+  uint16_t* zs = reinterpret_cast<uint16_t*>(zs4);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    no_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar, (uint32_t)nvec * 16u);
+    if (nvec > 0) bulk_load_smem(zs4, zr + base, (uint32_t)nvec * 16u, &bar);
+  }
+  // the tail, padded with -inf to a whole vector
+  if (tail && (int)threadIdx.x < 8) {
+    const int c = nvec * 8 + (int)threadIdx.x;
+    zs[c] = c < n ? reinterpret_cast<const uint16_t*>(zr)[base + c] : (uint16_t)0xff80u;
+  }
+  if (!mbar_wait(&bar, 0, &no_abort, err)) {
+    // the copy did not land within the wait limit: the error word says so; every
+    // thread still takes every barrier below, so the cluster is not held up
+  }
+  __syncthreads();
+  const float zt = (threadIdx.x == 0 && owns_t) ? __bfloat162float(__ushort_as_bfloat16(zs[t - base])) : 0.f;
+  __nv_bfloat162 m2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
+  for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
+    const uint4 u = zs4[v];
+    m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.z));
+    m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.w));
+  }
+  float m = fmaxf(__low2float(m2), __high2float(m2));
+  m = block_reduce_256(m, true, red);
+  const float ms = m == -INFINITY ? 0.f : m * LOG2E_F;  // an all -inf slice sums to 0
+  float s = 0.f;
+  for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
+    const uint4 u = zs4[v];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      s += ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ms)) + ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ms));
+  }
+  s = block_reduce_256(s, false, red);
+  if (threadIdx.x == 0) {
+    const uint32_t slot = smem_u32(&parts[rank]);
+    for (uint32_t q = 0; q < csize; ++q) st_cluster_f32x2(mapa_shared(slot, q), m, s);
+  }
+  cluster_sync();  // every CTA now holds all pairs; no CTA touches a peer after this
+  float M = -INFINITY;
+  for (uint32_t q = 0; q < csize; ++q) M = fmaxf(M, parts[q].x);
+  float S = 0.f;
+  for (uint32_t q = 0; q < csize; ++q)
+    if (parts[q].x != -INFINITY) S += parts[q].y * exp2f((parts[q].x - M) * LOG2E_F);
+  const float lse = M + logf(S);
+  if (threadIdx.x == 0) {
+    if (owns_t) a.row_loss[r] = lse - zt;
+    if (!valid && rank == 0) a.row_loss[r] = 0.f;
+    if (a.lse_out && rank == 0) a.lse_out[r] = lse;
+  }
+  if (!a.dz) return;
+  // 0 for ignored rows: every dz of such a row is exp(.) * 0 = 0
+  const float scale = valid ? mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f) : 0.f;
+  const float ls = lse * LOG2E_F;
+  const int tl = owns_t ? t - base : -1;  // the target's column within the slice
+  for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
+    const uint4 u = zs4[v];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float d0 = ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ls)) * scale;
+      float d1 = ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ls)) * scale;
+      if (v * 8 + 2 * q == tl) d0 -= scale;
+      if (v * 8 + 2 * q + 1 == tl) d1 -= scale;
+      o[q] = pack_bf16x2(d0, d1);
+    }
+    zs4[v] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
+  fence_proxy_async_smem();  // this thread's writes, before the bulk copy reads them
+  __syncthreads();
+  if (tail && (int)threadIdx.x < tail) {
+    const int c = nvec * 8 + (int)threadIdx.x;
+    reinterpret_cast<uint16_t*>(dr)[base + c] = zs[c];
+  }
+  if (threadIdx.x == 0 && nvec > 0) {
+    bulk_store_global(dr + base, zs4, (uint32_t)nvec * 16u);
+    bulk_commit_group();
+    bulk_wait_group_all();  // the shared memory it reads stays allocated until the copy is done
+  }
+}
+
 // ------------------------------------------------------------------ loss
 // One block, fixed order: thread k sums rows k, k+1024, ... in double, then a
 // fixed shuffle tree. Deterministic for a given BT.

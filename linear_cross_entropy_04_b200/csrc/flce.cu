@@ -114,7 +114,9 @@ flce_status device_ctx(DeviceCtx** out) {
       // non-portable size) when the device can hold one, else up to 8.
       c.ce_max_cluster = 8;
       if (cudaFuncSetAttribute(ce_row_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-          cudaSuccess) {
+              cudaSuccess &&
+          cudaFuncSetAttribute(ce_row_smem_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+              cudaSuccess) {
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
         cudaLaunchAttribute attr;
@@ -126,9 +128,12 @@ flce_status device_ctx(DeviceCtx** out) {
         cfg.blockDim = dim3(CER_THREADS);
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        int nc = 0;
-        if (cudaOccupancyMaxActiveClusters(&nc, ce_row_cluster_kernel, &cfg) == cudaSuccess && nc > 0)
-          c.ce_max_cluster = CER_MAX_CLUSTER;
+        int nc = 0, nc2 = 0;
+        if (cudaOccupancyMaxActiveClusters(&nc, ce_row_cluster_kernel, &cfg) == cudaSuccess && nc > 0) {
+          cfg.dynamicSmemBytes = CER_SLICE * 2;
+          if (cudaOccupancyMaxActiveClusters(&nc2, ce_row_smem_kernel, &cfg) == cudaSuccess && nc2 > 0)
+            c.ce_max_cluster = CER_MAX_CLUSTER;
+        }
       }
       cudaGetLastError();
       // Load the upstream-gradient kernels now: under lazy module loading a
@@ -482,6 +487,13 @@ Engine engine() {
 bool ce_one_pass_enabled() {
   const char* s = std::getenv("FLCE_CE");
   return !(s && std::strcmp(s, "multipass") == 0);
+}
+
+// FLCE_CE=regs keeps the one-pass CE slice in registers (ce_row_cluster_kernel)
+// instead of staging it in shared memory (ce_row_smem_kernel, the default).
+bool ce_slice_in_registers() {
+  const char* s = std::getenv("FLCE_CE");
+  return s && std::strcmp(s, "regs") == 0;
 }
 
 // Share of `units` workers kept busy over the waves of `tiles` equal tiles.
@@ -1145,10 +1157,12 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
                   grad ? grad->stride[0] : 0, tgt + r0, ignore_index, V, rl + r0,
                   (opt && opt->lse) ? opt->lse + r0 : nullptr, nv, reduction, row_grad ? row_grad + r0 : nullptr,
                   slice};
+      const bool regs = ce_slice_in_registers();
       st = L.run(1, [&] {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)cer_c, (unsigned)rows, 1);
         cfg.blockDim = dim3(CER_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = regs ? 0 : (size_t)slice * 2;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1157,7 +1171,10 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        cudaLaunchKernelEx(&cfg, ce_row_cluster_kernel, a);
+        if (regs)
+          cudaLaunchKernelEx(&cfg, ce_row_cluster_kernel, a);
+        else
+          cudaLaunchKernelEx(&cfg, ce_row_smem_kernel, a, dev->err);
       });
       if (st != FLCE_OK) return st;
     }

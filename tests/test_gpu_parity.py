@@ -432,17 +432,44 @@ def test_cross_entropy_one_pass_edge_rows():
     assert_grad_close(dz, ref["dz"], "bf16", "dz (-inf)")
 
 
-def test_cross_entropy_one_pass_matches_multipass(monkeypatch):
-    """The one-pass cluster kernel and the partials + combine + grad kernels agree."""
-    z, t = _ce_inputs(9, 256, 128256)
-    zd, td = z.cuda(), torch.from_numpy(t).cuda()
-    l1, g1 = L().cross_entropy(zd, td)
-    monkeypatch.setenv("FLCE_CE", "multipass")
-    l2, g2 = L().cross_entropy(zd, td)
-    torch.cuda.synchronize()
-    assert rel_err(l1.item(), l2.item()) <= 1e-5
-    d = (g1.float() - g2.float()).abs().max().item()
-    assert d <= 2 ** -8 * g2.float().abs().max().item(), d
+@pytest.mark.parametrize("V", [128256, 50021, 16391, 7])
+def test_cross_entropy_one_pass_matches_multipass(monkeypatch, V):
+    """The one-pass kernels (slice staged in shared memory, the default, and slice in
+    registers, FLCE_CE=regs) agree with the oracle, with the partials + combine + grad
+    kernels, and with each other bit for bit (same arithmetic in the same order).
+    Ragged V leaves a tail of fewer than 8 columns in the last CTA's slice; rows are
+    padded to 16 bytes and the padding columns must stay untouched."""
+    import ctypes
+
+    from linear_cross_entropy_04_b200 import _binding as B
+
+    Vp = V + (-V) % 8
+    z, t = _ce_inputs(9, 256, V)
+    zp = torch.full((256, Vp), -1.0, dtype=torch.bfloat16)
+    zp[:, :V] = z
+    zd, td = zp.cuda()[:, :V], torch.from_numpy(t).cuda()
+    assert zd.stride(0) == Vp
+    gp = torch.full((256, Vp), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = {}
+    for mode in ("", "regs", "multipass"):
+        if mode:
+            monkeypatch.setenv("FLCE_CE", mode)
+        g = gp[:, :V]
+        loss = torch.empty((), dtype=torch.float32, device="cuda")
+        tz, tt, tl, tg = B.tensor(zd), B.tensor(td), B.tensor(loss), B.tensor(g)
+        B.check(B.lib().flce_cross_entropy(ctypes.byref(tz), ctypes.byref(tt), -100, 0, ctypes.byref(tl),
+                                           ctypes.byref(tg), B.stream_handle(), None), "flce_cross_entropy")
+        torch.cuda.synchronize()
+        assert L().device_error() == 0
+        assert torch.all(gp[:, V:] == 7.0), "padding columns must stay untouched"
+        out[mode] = (loss.item(), g.clone())
+    ref = oracle.cross_entropy(z.double().numpy(), t)
+    for mode, (lv, g) in out.items():
+        assert rel_err(lv, ref["loss"]) <= TOL["bf16"]["loss"], mode
+        assert_grad_close(g, ref["dz"], "bf16", f"dz ({mode or 'smem'})")
+    assert out[""][0] == out["regs"][0] and torch.equal(out[""][1], out["regs"][1])
+    d = (out[""][1].float() - out["multipass"][1].float()).abs().max().item()
+    assert d <= 2 ** -8 * out["multipass"][1].float().abs().max().item(), d
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
