@@ -211,10 +211,13 @@ def test_module_backward_does_not_wait_for_the_gpu():
     gradients still come out scaled (1 leaves them untouched, 0.5 halves them)."""
     d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=256, H=128, V=1000)
     ref = oracle.flce(d["X"], d["W"], d["target"])
-    # one untimed backward first: under lazy module loading the first launch of any kernel
-    # in the process (torch's own included) may block the host once
-    X, W, t = to_dev(d)
-    L().FusedLinearCrossEntropyLoss()(W.requires_grad_(True), X.requires_grad_(True), t).backward()
+    # the same sequence untimed first: under lazy module loading the first launch of any
+    # kernel in the process (torch's own included, such as the multiply's backward) may
+    # block the host once
+    for factor in (1.0, 0.5):
+        X, W, t = to_dev(d)
+        loss = L().FusedLinearCrossEntropyLoss()(W.requires_grad_(True), X.requires_grad_(True), t)
+        (loss * factor).backward()
     torch.cuda.synchronize()
     for factor in (1.0, 0.5):
         X, W, t = to_dev(d)
@@ -436,7 +439,8 @@ def test_cross_entropy_one_pass_edge_rows():
 def test_cross_entropy_one_pass_matches_multipass(monkeypatch, V):
     """The one-pass kernels (slice staged in shared memory, the default, and slice in
     registers, FLCE_CE=regs) agree with the oracle, with the partials + combine + grad
-    kernels, and with each other bit for bit (same arithmetic in the same order).
+    kernels, and with each other to bf16 rounding (their reductions merge in
+    different orders).
     Ragged V leaves a tail of fewer than 8 columns in the last CTA's slice; rows are
     padded to 16 bytes and the padding columns must stay untouched."""
     import ctypes
@@ -467,9 +471,10 @@ def test_cross_entropy_one_pass_matches_multipass(monkeypatch, V):
     for mode, (lv, g) in out.items():
         assert rel_err(lv, ref["loss"]) <= TOL["bf16"]["loss"], mode
         assert_grad_close(g, ref["dz"], "bf16", f"dz ({mode or 'smem'})")
-    assert out[""][0] == out["regs"][0] and torch.equal(out[""][1], out["regs"][1])
-    d = (out[""][1].float() - out["multipass"][1].float()).abs().max().item()
-    assert d <= 2 ** -8 * out["multipass"][1].float().abs().max().item(), d
+    for other in ("regs", "multipass"):
+        assert rel_err(out[""][0], out[other][0]) <= 1e-5, other
+        d = (out[""][1].float() - out[other][1].float()).abs().max().item()
+        assert d <= 2 ** -8 * out[other][1].float().abs().max().item(), (other, d)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
