@@ -650,7 +650,9 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
     // the copy did not land within the wait limit: the error word says so; every
     // thread still takes every barrier below, so the cluster is not held up
   }
-  // this thread's (max, sum of exp(z - max)) over its vectors, then one block merge
+  // the warp's max over its threads' vectors (shuffles, no block barrier), each
+  // thread's sum of exp(z - warp max), the warp's sum, then one block merge of
+  // the 8 warps' (max, sum) pairs
   __nv_bfloat162 m2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
   float zt = 0.f;
   for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
@@ -662,8 +664,10 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
     if ((tl >> 3) == v) zt = __bfloat162float(__ushort_as_bfloat16(reinterpret_cast<const uint16_t*>(zs4)[tl]));
   }
   float m = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float s = 0.f;
-  if (m != -INFINITY) {
+  if (m != -INFINITY) {  // warp-uniform
     const float ms = m * LOG2E_F;
     for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
       const uint4 u = zs4[v];
@@ -674,10 +678,7 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float mo = __shfl_xor_sync(0xffffffffu, m, o), so = __shfl_xor_sync(0xffffffffu, s, o);
-    merge_max_sum(m, s, mo, so);
-  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(m, s);
   __syncthreads();
   if (threadIdx.x == 0) {
