@@ -585,17 +585,9 @@ __device__ __forceinline__ void bulk_store_global(void* gdst, const void* smem_s
                : "memory");
 }
 
-// Merge two (max, sum of exp(x - max)) pairs; an empty pair is (-inf, 0).
-__device__ __forceinline__ void merge_max_sum(float& m, float& s, float m2, float s2) {
-  const float M = fmaxf(m, m2);
-  if (M == -INFINITY) return;
-  s = (m == -INFINITY ? 0.f : s * exp2f((m - M) * LOG2E_F)) + (m2 == -INFINITY ? 0.f : s2 * exp2f((m2 - M) * LOG2E_F));
-  m = M;
-}
-
 __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, uint32_t* err) {
   extern __shared__ __align__(128) uint4 zs4[];  // the slice: (slice / 8) 16-byte vectors
-  __shared__ float2 red[CER_THREADS / 32];
+  __shared__ float red[CER_THREADS / 32];
   __shared__ float2 parts[CER_MAX_CLUSTER];
   __shared__ __align__(8) uint64_t bar;
   __shared__ int no_abort;
@@ -611,7 +603,7 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
   const int64_t t64 = a.target[r];
   const bool valid = target_valid(t64, a.V, a.ignore_index);
   const int t = valid ? (int)t64 : -1;
-  const int tl = valid && t >= base && t < end ? t - base : -1;  // the target's column in this slice
+  const bool owns_t = valid && t >= base && t < end;
   if (!valid && !a.lse_out) {
     // an ignored row needs neither its logits nor a cluster exchange (every CTA of
     // the cluster takes this branch: they share the row)
@@ -628,6 +620,7 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
     }
     return;
   }
+  uint16_t* zs = reinterpret_cast<uint16_t*>(zs4);
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     no_abort = 0;
@@ -638,55 +631,40 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
     mbar_arrive_expect_tx(&bar, (uint32_t)nvec * 16u);
     if (nvec > 0) bulk_load_smem(zs4, zr + base, (uint32_t)nvec * 16u, &bar);
   }
-  // the partial last vector (V not a multiple of 8): read by the thread that owns it,
-  // padded with -inf, and kept in shared memory for that thread's later passes
-  if (tail && (nvec & (CER_THREADS - 1)) == (int)threadIdx.x) {
-    uint16_t* zs = reinterpret_cast<uint16_t*>(zs4);
-    const uint16_t* zb = reinterpret_cast<const uint16_t*>(zr) + base;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) zs[nvec * 8 + k] = k < tail ? zb[nvec * 8 + k] : (uint16_t)0xff80u;
+  // the tail, padded with -inf to a whole vector
+  if (tail && (int)threadIdx.x < 8) {
+    const int c = nvec * 8 + (int)threadIdx.x;
+    zs[c] = c < n ? reinterpret_cast<const uint16_t*>(zr)[base + c] : (uint16_t)0xff80u;
   }
   if (!mbar_wait(&bar, 0, &no_abort, err)) {
     // the copy did not land within the wait limit: the error word says so; every
     // thread still takes every barrier below, so the cluster is not held up
   }
-  // the warp's max over its threads' vectors (shuffles, no block barrier), each
-  // thread's sum of exp(z - warp max), the warp's sum, then one block merge of
-  // the 8 warps' (max, sum) pairs
+  __syncthreads();
+  const float zt = (threadIdx.x == 0 && owns_t) ? __bfloat162float(__ushort_as_bfloat16(zs[t - base])) : 0.f;
   __nv_bfloat162 m2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
-  float zt = 0.f;
   for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
     const uint4 u = zs4[v];
     m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.x));
     m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.y));
     m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.z));
     m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&u.w));
-    if ((tl >> 3) == v) zt = __bfloat162float(__ushort_as_bfloat16(reinterpret_cast<const uint16_t*>(zs4)[tl]));
   }
   float m = fmaxf(__low2float(m2), __high2float(m2));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  m = block_reduce_256(m, true, red);
+  const float ms = m == -INFINITY ? 0.f : m * LOG2E_F;  // an all -inf slice sums to 0
   float s = 0.f;
-  if (m != -INFINITY) {  // warp-uniform
-    const float ms = m * LOG2E_F;
-    for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
-      const uint4 u = zs4[v];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
+    const uint4 u = zs4[v];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        s += ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ms)) + ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ms));
-    }
+    for (int q = 0; q < 4; ++q)
+      s += ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ms)) + ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ms));
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(m, s);
-  __syncthreads();
+  s = block_reduce_256(s, false, red);
   if (threadIdx.x == 0) {
-    float mb = red[0].x, sb = red[0].y;
-#pragma unroll
-    for (int k = 1; k < CER_THREADS / 32; ++k) merge_max_sum(mb, sb, red[k].x, red[k].y);
     const uint32_t slot = smem_u32(&parts[rank]);
-    for (uint32_t q = 0; q < csize; ++q) st_cluster_f32x2(mapa_shared(slot, q), mb, sb);
+    for (uint32_t q = 0; q < csize; ++q) st_cluster_f32x2(mapa_shared(slot, q), m, s);
   }
   cluster_sync();  // every CTA now holds all pairs; no CTA touches a peer after this
   float M = -INFINITY;
@@ -695,16 +673,16 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
   for (uint32_t q = 0; q < csize; ++q)
     if (parts[q].x != -INFINITY) S += parts[q].y * exp2f((parts[q].x - M) * LOG2E_F);
   const float lse = M + logf(S);
-  if (tl >= 0 && (tl >> 3) % CER_THREADS == (int)threadIdx.x) a.row_loss[r] = lse - zt;
-  if (threadIdx.x == 0 && rank == 0) {
-    if (!valid) a.row_loss[r] = 0.f;
-    if (a.lse_out) a.lse_out[r] = lse;
+  if (threadIdx.x == 0) {
+    if (owns_t) a.row_loss[r] = lse - zt;
+    if (!valid && rank == 0) a.row_loss[r] = 0.f;
+    if (a.lse_out && rank == 0) a.lse_out[r] = lse;
   }
   if (!a.dz) return;
   // 0 for ignored rows: every dz of such a row is exp(.) * 0 = 0
   const float scale = valid ? mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f) : 0.f;
   const float ls = lse * LOG2E_F;
-  __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
+  const int tl = owns_t ? t - base : -1;  // the target's column within the slice
   for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
     const uint4 u = zs4[v];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -717,20 +695,15 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
       if (v * 8 + 2 * q + 1 == tl) d1 -= scale;
       o[q] = pack_bf16x2(d0, d1);
     }
-    if (v < nvec) {
-      zs4[v] = make_uint4(o[0], o[1], o[2], o[3]);
-    } else {
-      // the partial last vector goes out by plain stores, from this thread
-      uint16_t* db = reinterpret_cast<uint16_t*>(dr) + base + v * 8;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (2 * q < tail) db[2 * q] = (uint16_t)(o[q] & 0xffffu);
-        if (2 * q + 1 < tail) db[2 * q + 1] = (uint16_t)(o[q] >> 16);
-      }
-    }
+    zs4[v] = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
   fence_proxy_async_smem();  // this thread's writes, before the bulk copy reads them
   __syncthreads();
+  if (tail && (int)threadIdx.x < tail) {
+    const int c = nvec * 8 + (int)threadIdx.x;
+    reinterpret_cast<uint16_t*>(dr)[base + c] = zs[c];
+  }
   if (threadIdx.x == 0 && nvec > 0) {
     bulk_store_global(dr + base, zs4, (uint32_t)nvec * 16u);
     bulk_commit_group();
