@@ -33,6 +33,10 @@
 namespace flce {
 
 __device__ uint32_t g_err_word;  // device error word (FLCE_DEVERR_* bits), one per device
+// checkpoint counters of the wide grad_X tiles' soft K-synchronisation (zeroed
+// before each launch that uses them; launches that overlap on the GPU only
+// disturb each other's pacing, not their results)
+__device__ uint32_t g_ksync_ctr[KSYNC_MAX_CKPT];
 
 namespace {
 
@@ -49,6 +53,7 @@ struct DeviceCtx {
   int pairs = 0;  // CTA pairs of the cluster engine that fit on the device at once
   int ce_max_cluster = 0;  // largest cluster the one-pass cross-entropy kernel can launch with
   uint32_t* err = nullptr;
+  uint32_t* ksync = nullptr;     // device address of g_ksync_ctr
   cudaMemPool_t pool = nullptr;  // library-owned stream-ordered pool for workspaces
 };
 
@@ -79,7 +84,8 @@ flce_status device_ctx(DeviceCtx** out) {
     c.supported = prop.major == 10 && prop.minor == 0;
     c.sms = prop.multiProcessorCount;
     if (c.supported) {
-      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.err), g_err_word) != cudaSuccess)
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.err), g_err_word) != cudaSuccess ||
+          cudaGetSymbolAddress(reinterpret_cast<void**>(&c.ksync), g_ksync_ctr) != cudaSuccess)
         return FLCE_ERR_CUDA;
       if (cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TC_SMEM_BYTES) != cudaSuccess ||
@@ -513,6 +519,12 @@ bool gradx_wide(int64_t tiles_m, int64_t N, int64_t units) {
   const double en = wave_efficiency(tiles_m * ceil_div(N, 256), units);
   const double ew = wave_efficiency(tiles_m * ceil_div(N, 512), units);
   return ew >= en - 1e-9;
+}
+
+// FLCE_KSYNC=0 turns off the soft K-synchronisation of one-wave wide grad_X tiles.
+bool ksync_enabled() {
+  const char* s = std::getenv("FLCE_KSYNC");
+  return !(s && s[0] == '0');
 }
 
 bool grad_combined(int64_t gradx_tiles, int64_t units) {
@@ -955,6 +967,14 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         if (eg.pair && gx_split == 1 && gradx_wide(P.tiles_m, H, dev->pairs)) {
           gx_wide = true;
           P.tiles_n = (int)ceil_div(H, T2W_BN);
+          // one wave of wide tiles: keep the pairs in step along K (counters zeroed first)
+          const int64_t wide_tiles = (int64_t)P.tiles_m * P.tiles_n;
+          const int64_t ckpts = P.kblocks / KSYNC_EVERY + 1;
+          if (wide_tiles <= dev->pairs && ckpts <= KSYNC_MAX_CKPT && ksync_enabled()) {
+            if (cudaMemsetAsync(dev->ksync, 0, (size_t)ckpts * 4, stream) != cudaSuccess) return FLCE_ERR_CUDA;
+            prm.kprog = dev->ksync;
+            prm.ksync_pairs = (int)wide_tiles;
+          }
         }
         prm.prob[np++] = P;
       }
@@ -1012,6 +1032,8 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         p2.nprob = 1;
         p2.prob[0] = prm.prob[1];
         p2.prob[1] = TcProblem{};
+        p2.kprog = nullptr;  // the K-synchronisation is grad_X's
+        p2.ksync_pairs = 0;
         CUtensorMap z;
         std::memset(&z, 0, sizeof(z));
         st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0], nullptr, nullptr, gx_wide); });

@@ -112,6 +112,14 @@ struct TcParams {
   // its output tile number test_stall - 1, on a barrier nothing arrives on, so the
   // bounded wait runs out and the kernel takes its abort path.
   int test_stall;
+  // Wide tiles in one wave: pairs [0, ksync_pairs) count their arrivals at every
+  // KSYNC_EVERY-th K-block in kprog[checkpoint] (zeroed before the launch), and a
+  // pair waits a bounded time at a checkpoint until every pair has passed the one
+  // KSYNC_WINDOW K-blocks back, so that the dz and W panels the tiles share stay
+  // in L2 between their readers. 0 = off. A performance hint only: nothing
+  // depends on it for correctness.
+  uint32_t* kprog;
+  int ksync_pairs;
 };
 
 // ------------------------------------------------------------ tile schedule

@@ -69,6 +69,25 @@ constexpr int T2W_B_BYTES = 2 * T2_B_BYTES;  // 32 KB
 constexpr int T2W_STAGE_BYTES = T2_A_BYTES + T2W_B_BYTES;
 constexpr int T2W_SMEM_BYTES = T2W_STAGES * T2W_STAGE_BYTES + T2_OUT_BYTES + 1024 + 256;
 
+// Soft K-synchronisation of one-wave wide tiles (TcParams::kprog): at every
+// KSYNC_EVERY-th K-block a pair adds one to that checkpoint's counter, then waits
+// until every synchronised pair has passed the checkpoint KSYNC_WINDOW K-blocks
+// back (at most KSYNC_CAP_NS; after a wait that runs out the pair stops
+// synchronising for the rest of the launch). One counter load per check.
+constexpr int KSYNC_EVERY = 16;
+#ifndef FLCE_KSYNC_WINDOW
+#define FLCE_KSYNC_WINDOW 64
+#endif
+constexpr int KSYNC_LAG = FLCE_KSYNC_WINDOW / KSYNC_EVERY;  // checkpoints of lead allowed (64 K-blocks: ~50 MB)
+constexpr int KSYNC_MAX_CKPT = 4096;                         // counters available (V up to 4M columns)
+constexpr uint64_t KSYNC_CAP_NS = 20000;
+
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // The epilogue of the first half of a wide tile hands nothing back yet.
 struct NoRelease {
   __device__ __forceinline__ void operator()() const {}
@@ -376,6 +395,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     if (lane == 0) {
       uint32_t kit = 0;
       bool ok = true;
+      // the leader's producer keeps its pair in step (the peer's follows through the MMA commits)
+      bool ksync = kWide && leader && p.kprog != nullptr && pair < p.ksync_pairs &&
+                   p.prob[0].kblocks / KSYNC_EVERY < KSYNC_MAX_CKPT;
       for (int i = 0; i < ntiles && ok; ++i) {
         const Tile T = sched_tile(p, sched, pair, G, i);
         const int pi = T.prob, tm = T.tm, tn = T.tn;
@@ -385,6 +407,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         const int am0 = tm * T2_BM + (int)rank * T2_HALF;  // this CTA's rows of A
         const int bn0 = tn * TILE_N + (int)rank * T2_HALF;  // this CTA's rows of B (wide: and bn0 + 256)
         for (int kb = T.kb0; kb < T.kb1; ++kb, ++kit) {
+          if (kWide && ksync && (kb % KSYNC_EVERY) == 0) {
+            // arrive at this checkpoint, then hold back while a pair is still KSYNC_LAG checkpoints behind
+            const int c = kb / KSYNC_EVERY;
+            atomicAdd(p.kprog + c, 1u);
+            if (c >= KSYNC_LAG) {
+              const uint32_t* behind = p.kprog + (c - KSYNC_LAG);
+              const uint64_t t0 = globaltimer_ns();
+              while (ld_relaxed_gpu(behind) < (uint32_t)p.ksync_pairs) {
+                if (globaltimer_ns() - t0 > KSYNC_CAP_NS || *abort_flag) {
+                  ksync = false;
+                  break;
+                }
+                __nanosleep(256);
+              }
+            }
+          }
           const int stage = kit % STAGES;
           const uint32_t phase = (kit / STAGES) & 1;
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
