@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define FLCE_VERSION 100 /* 1.0.0 */
+#define FLCE_VERSION 110 /* 1.1.0: flce_scale_grad, flce_gemm_bf16_wait_test, FLCE_FLAG_RECOMPUTE, FLCE_FLAG_ROUTE_EVERY_CHUNK */
 
 #if defined(__GNUC__)
 #define FLCE_API __attribute__((visibility("default")))

@@ -46,7 +46,7 @@ def test_binding_signatures_cover_the_header():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.flce_version() == 100
+    assert lib.flce_version() == 110
     assert lib.flce_status_string(0) == b"ok"
     assert b"unsupported device" in lib.flce_status_string(3)
     assert lib.flce_status_string(99) == b"unknown status"
