@@ -176,11 +176,16 @@ typedef struct {
   int32_t path;                      /* 0 = SIMT fp32 path, 1 = tcgen05 bf16 path */
 } flce_stats;
 
-/* Fill *opt with the defaults (all zero / NULL). */
+/* Fill *opt with the defaults (all zero / NULL). Library infrastructure: no passage of the pages
+ * defines it. */
 FLCE_API void flce_options_init(flce_options* opt);
 
 /*
- * Fused linear cross-entropy, forward and backward, in one call.
+ * Fused linear cross-entropy, forward and backward, in one call: the chunked fused
+ * Linear + CrossEntropy of "Liger Kernel: Efficient Triton Kernels for LLM Training"
+ * (paper review, 提案手法; Figure 1), called as the low-level API of "Liger-Kernel
+ * 項目詳細介紹" (使用方法 > 3. 低級 API 方式) is: loss_fn(weight, input, target), then
+ * loss.backward(). The operation is the one this header's preamble writes out.
  *   X       [BT,H]  bf16 or f32 (row-major)
  *   W       [V,H]   same dtype as X
  *   target  [BT]    int64; rows equal to ignore_index are ignored
@@ -206,7 +211,8 @@ FLCE_API flce_status flce_fwd_bwd_ex(const flce_tensor* X, const flce_tensor* W,
                             flce_stream_t stream, const flce_options* opt, flce_stats* stats);
 
 /*
- * Host-only planning: fills *out with the chunk rows, chunk count and
+ * Host-only planning (the chunking of "Liger-Kernel 項目詳細介紹", 技術原理 > 分塊計算,
+ * sized for a workspace budget): fills *out with the chunk rows, chunk count and
  * workspace bytes flce_fwd_bwd_ex would use for this shape. Touches no GPU.
  * dtype is FLCE_BF16 or FLCE_F32. want_grad_W selects whether a grad_W
  * accumulator (FLCE_GRADW_ACCUM_FP32) is counted.
@@ -215,6 +221,7 @@ FLCE_API flce_status flce_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, 
                       const flce_options* opt, flce_stats* out);
 
 /*
+ * Library infrastructure (no passage defines it; it sizes the chunking's memory).
  * Host-only: the workspace bytes flce_fwd_bwd_ex would use for this shape and
  * options with grad_W requested (flce_plan's workspace_bytes), i.e. the size a
  * caller-provided opt->workspace needs. 0 for an empty batch; (size_t)-1 if
@@ -223,7 +230,8 @@ FLCE_API flce_status flce_plan(int64_t BT, int64_t H, int64_t V, int32_t dtype, 
 FLCE_API size_t flce_workspace_bytes(int64_t BT, int64_t H, int64_t V, int32_t dtype, const flce_options* opt);
 
 /*
- * N, the count of rows whose target is not ignore_index, written as int64
+ * The mean's denominator: N, the count of rows whose target is not ignore_index (the
+ * ignore_index of the low-level API, "Liger-Kernel 項目詳細介紹", 使用方法 > 3), written as int64
  * to the DEVICE pointer n_valid_out on `stream`. Targets outside [0,V) that
  * are not ignore_index set FLCE_DEVERR_TARGET_RANGE and are not counted.
  * Used by data-parallel callers to all-reduce N before flce_fwd_bwd_ex.
@@ -282,7 +290,8 @@ FLCE_API flce_status flce_cross_entropy_noalloc(const flce_tensor* logits, const
                                                 flce_tensor* grad_logits, flce_stream_t stream);
 
 /*
- * Plain bf16 GEMM on the library's tcgen05 engine, for testing that engine
+ * Test hook; no passage defines it (the pages' method runs its contractions inside the
+ * fused call). Plain bf16 GEMM on the library's tcgen05 engine, for testing that engine
  * on its own: C[M,N] (f32, row-major, ldc) = sum_k A(m,k) * B(n,k).
  * A is [M,K] row-major (a_mn_major = 0, lda >= K) or [K,M] row-major
  * (a_mn_major = 1, lda >= M); B likewise with N. Leading dimensions are in
@@ -328,6 +337,8 @@ FLCE_API flce_status flce_gemm_bf16_wait_test(const void* A, const void* B, floa
 FLCE_API flce_status flce_scale_grad(flce_tensor* t, const float* scale, flce_stream_t stream);
 
 /*
+ * Library infrastructure (no passage defines it): device-side data errors and
+ * wait timeouts are reported here instead of trapping.
  * Waits for `stream`, then returns the device error word of the current
  * device in *err (FLCE_DEVERR_* bits) and clears it. The word is shared by
  * every stream on the device.
@@ -335,6 +346,7 @@ FLCE_API flce_status flce_scale_grad(flce_tensor* t, const float* scale, flce_st
 FLCE_API flce_status flce_get_device_error(flce_stream_t stream, uint32_t* err);
 
 /*
+ * Library infrastructure (no passage defines it).
  * Phase timing (calls made with FLCE_FLAG_TIME_PHASES): waits for the
  * recorded events and writes, for each phase p < n_phases, the summed
  * milliseconds to ms[p] and the number of timed launches to count[p] (either
@@ -348,10 +360,10 @@ FLCE_API flce_status flce_get_device_error(flce_stream_t stream, uint32_t* err);
 #define FLCE_NUM_PHASES 6
 FLCE_API flce_status flce_phase_times(double* ms, int32_t* count, int32_t n_phases, int32_t reset);
 
-/* Static string for a status code. */
+/* Static string for a status code. Library infrastructure: no passage defines it. */
 FLCE_API const char* flce_status_string(int32_t status);
 
-/* FLCE_VERSION of the built library. */
+/* FLCE_VERSION of the built library. Library infrastructure: no passage defines it. */
 FLCE_API int32_t flce_version(void);
 
 #ifdef __cplusplus
