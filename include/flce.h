@@ -183,9 +183,9 @@ FLCE_API void flce_options_init(flce_options* opt);
 /*
  * Fused linear cross-entropy, forward and backward, in one call: the chunked fused
  * Linear + CrossEntropy of "Liger Kernel: Efficient Triton Kernels for LLM Training"
- * (paper review, 提案手法; Figure 1), called as the low-level API of "Liger-Kernel
- * 項目詳細介紹" (使用方法 > 3. 低級 API 方式) is: loss_fn(weight, input, target), then
- * loss.backward(). The operation is the one this header's preamble writes out.
+ * (paper review, 提案手法; Figure 1), with the call shape of the low-level API of
+ * "Liger-Kernel 項目詳細介紹" (使用方法 > 3. 低級 API 方式): loss_fn(weight, input, target),
+ * then loss.backward(). The operation is the one this header's preamble writes out.
  *   X       [BT,H]  bf16 or f32 (row-major)
  *   W       [V,H]   same dtype as X
  *   target  [BT]    int64; rows equal to ignore_index are ignored
