@@ -44,7 +44,8 @@ constexpr int kMaxDevices = 64;
 constexpr int64_t kDefaultLimit = 512ll << 20;
 constexpr int64_t kMaxChunk = 32768;
 constexpr int64_t kMinDefaultChunk = 2048;
-constexpr int64_t kRecomputeRowBlock = 4096;  // rows per logits launch in the recompute schedule's first pass
+constexpr int64_t kRecomputeRowBlock = 4096;
+constexpr int kCeSliceMax = 32768;  // largest slice of the shared-memory one-pass CE kernel (64 KB staged)  // rows per logits launch in the recompute schedule's first pass
 
 struct DeviceCtx {
   bool init = false;
@@ -119,6 +120,9 @@ flce_status device_ctx(DeviceCtx** out) {
       // The one-pass cross-entropy kernel runs clusters of up to 16 CTAs (a
       // non-portable size) when the device can hold one, else up to 8.
       c.ce_max_cluster = 8;
+      if (cudaFuncSetAttribute(ce_row_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCeSliceMax * 2) !=
+          cudaSuccess)
+        return FLCE_ERR_CUDA;
       if (cudaFuncSetAttribute(ce_row_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
               cudaSuccess &&
           cudaFuncSetAttribute(ce_row_smem_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
@@ -500,6 +504,18 @@ bool ce_one_pass_enabled() {
 bool ce_slice_in_registers() {
   const char* s = std::getenv("FLCE_CE");
   return s && std::strcmp(s, "regs") == 0;
+}
+
+// Columns per CTA of the shared-memory one-pass kernel (FLCE_CE_SLICE, a multiple
+// of 8 in [2048, 32768]; default 16384): the slice is staged in slice * 2 bytes of
+// shared memory, and a row takes ceil(V / slice) CTAs (at most 16).
+int ce_slice_cols() {
+  const char* s = std::getenv("FLCE_CE_SLICE");
+  if (!s || !*s) return CER_SLICE;
+  char* end = nullptr;
+  const long v = std::strtol(s, &end, 10);
+  if (end == s || *end != '\0' || v < 2048 || v > kCeSliceMax || v % 8) return CER_SLICE;
+  return (int)v;
 }
 
 // Share of `units` workers kept busy over the waves of `tiles` equal tiles.
@@ -1141,9 +1157,10 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
     return cudaMemsetAsync(loss->data, 0, 4, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
   }
   const int shift = 10;
-  // bf16 rows up to CER_SLICE * (largest cluster) columns take the one-pass
-  // cluster kernel, which needs no partials; the rest take partials + combine + grad
-  const int cer_c = (int)ceil_div(V, CER_SLICE);
+  // bf16 rows up to (slice columns) * (largest cluster) take a one-pass cluster
+  // kernel, which needs no partials; the rest take partials + combine + grad
+  const bool regs = ce_slice_in_registers();
+  const int cer_c = (int)ceil_div(V, regs ? CER_SLICE : ce_slice_cols());
   const bool one_pass = dt == FLCE_BF16 && cer_c <= dev->ce_max_cluster && ce_one_pass_enabled();
   const int64_t ntile = one_pass ? 0 : ceil_div(V, 1 << shift), ldp = round_up(BT, 32);
   size_t o = 0;
@@ -1179,7 +1196,6 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
                   grad ? grad->stride[0] : 0, tgt + r0, ignore_index, V, rl + r0,
                   (opt && opt->lse) ? opt->lse + r0 : nullptr, nv, reduction, row_grad ? row_grad + r0 : nullptr,
                   slice};
-      const bool regs = ce_slice_in_registers();
       st = L.run(1, [&] {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)cer_c, (unsigned)rows, 1);
