@@ -374,11 +374,11 @@ def run_ce(args):
         res[name] = {"ms_per_step": ms, "tokens_per_s": w.BT / (ms / 1e3),
                      "peak_extra_bytes": torch.cuda.max_memory_allocated(dev) - base, "clocks": clk.summary()}
     # the library's CE workspace (taken from its own pool, invisible to torch's counters).
-    # One-pass cluster kernel (bf16, V <= 16 * 16384): N and the per-row losses.
+    # One-pass cluster kernel (bf16, V <= 16 * 32768): N and the per-row losses.
     # Multi-pass kernels: also per-row lse / target logit and per-(1024-column
     # tile, row) max and sum-exp.
     a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
-    one_pass = w.dtype == "bf16" and w.V <= 16 * 16384 and os.environ.get("FLCE_CE") != "multipass"
+    one_pass = w.dtype == "bf16" and w.V <= 16 * 32768 and os.environ.get("FLCE_CE") != "multipass"
     if one_pass:
         lib_ws = a256(8) + a256(4 * w.BT)
     else:

@@ -247,10 +247,12 @@ FLCE_API flce_status flce_count_valid(const flce_tensor* target, int64_t V, int6
  *   logits tensor itself (in-place gradient replacement).
  * opt may be NULL; only opt->n_valid, opt->row_loss, opt->lse and opt->row_grad are read.
  * FLCE_NONE as for flce_fwd_bwd (loss is f32 [BT]).
- * bf16 logits with V up to 16 * 16384 (8 * 16384 on a device that cannot hold
+ * bf16 logits with V up to 16 * 32768 (8 * 32768 on a device that cannot hold
  * a 16-CTA cluster) take one pass: a thread-block cluster per row reads the
  * logits once and writes the gradient once, with a workspace of N and the
- * per-row losses only. f32 logits and longer rows take three passes (per-tile
+ * per-row losses only. Each CTA of the cluster stages its slice of the row in
+ * shared memory: ceil(V / 24576) CTAs up to 8, else slices of up to 32768
+ * columns (FLCE_CE_SLICE=<columns> sets the slice). f32 logits and longer rows take three passes (per-tile
  * partials, row combine, gradient) with a per-(row, 1024-column tile) partials
  * workspace. The workspace comes from the library's memory pool.
  */

@@ -140,7 +140,7 @@ flce_status device_ctx(DeviceCtx** out) {
         cfg.numAttrs = 1;
         int nc = 0, nc2 = 0;
         if (cudaOccupancyMaxActiveClusters(&nc, ce_row_cluster_kernel, &cfg) == cudaSuccess && nc > 0) {
-          cfg.dynamicSmemBytes = CER_SLICE * 2;
+          cfg.dynamicSmemBytes = kCeSliceMax * 2;  // the largest slice the shared-memory kernel stages
           if (cudaOccupancyMaxActiveClusters(&nc2, ce_row_smem_kernel, &cfg) == cudaSuccess && nc2 > 0)
             c.ce_max_cluster = CER_MAX_CLUSTER;
         }
@@ -506,16 +506,23 @@ bool ce_slice_in_registers() {
   return s && std::strcmp(s, "regs") == 0;
 }
 
-// Columns per CTA of the shared-memory one-pass kernel (FLCE_CE_SLICE, a multiple
-// of 8 in [2048, 32768]; default 16384): the slice is staged in slice * 2 bytes of
-// shared memory, and a row takes ceil(V / slice) CTAs (at most 16).
-int ce_slice_cols() {
+// CTAs per row (the cluster size) of the shared-memory one-pass CE kernel; each
+// stages ceil(V / C) columns, rounded up to 8, in shared memory (2 bytes each, at
+// most kCeSliceMax columns). Measured on B200 (4096 rows): clusters of 6-8 CTAs
+// with 3-5 CTAs per SM run fastest (V = 128256: 0.412 ms with 6 CTAs of 21376
+// columns, against 0.450 with 8 and 0.437 with 4; V = 256000: 0.898 ms with 8 of
+// 32000, against 0.973 with 11 and 0.970 with 16). So C = ceil(V / 24576), or, when
+// that is above 8, the larger of 8 and ceil(V / 32768). FLCE_CE_SLICE=<columns>
+// (a multiple of 8 in [2048, 32768]) sets the slice instead: C = ceil(V / slice).
+int64_t ce_smem_ctas(int64_t V) {
   const char* s = std::getenv("FLCE_CE_SLICE");
-  if (!s || !*s) return CER_SLICE;
-  char* end = nullptr;
-  const long v = std::strtol(s, &end, 10);
-  if (end == s || *end != '\0' || v < 2048 || v > kCeSliceMax || v % 8) return CER_SLICE;
-  return (int)v;
+  if (s && *s) {
+    char* end = nullptr;
+    const long v = std::strtol(s, &end, 10);
+    if (end != s && *end == '\0' && v >= 2048 && v <= kCeSliceMax && v % 8 == 0) return ceil_div(V, v);
+  }
+  const int64_t c = ceil_div(V, 24576);
+  return c <= 8 ? c : std::max<int64_t>(8, ceil_div(V, kCeSliceMax));
 }
 
 // Share of `units` workers kept busy over the waves of `tiles` equal tiles.
@@ -1160,7 +1167,8 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   // bf16 rows up to (slice columns) * (largest cluster) take a one-pass cluster
   // kernel, which needs no partials; the rest take partials + combine + grad
   const bool regs = ce_slice_in_registers();
-  const int cer_c = (int)ceil_div(V, regs ? CER_SLICE : ce_slice_cols());
+  const int64_t cer_c64 = regs ? ceil_div(V, CER_SLICE) : ce_smem_ctas(V);
+  const int cer_c = (int)std::min<int64_t>(cer_c64, 1 << 20);
   const bool one_pass = dt == FLCE_BF16 && cer_c <= dev->ce_max_cluster && ce_one_pass_enabled();
   const int64_t ntile = one_pass ? 0 : ceil_div(V, 1 << shift), ldp = round_up(BT, 32);
   size_t o = 0;

@@ -375,9 +375,11 @@ def _ce_inputs(seed, BT, V, ignore_every=6):
     return z, t
 
 
-# V spans one-pass clusters of 1, 2, 4, 8, 10 and 16 CTAs, and a V past the
-# largest cluster (and not a multiple of 8) that takes the multi-pass kernels.
-@pytest.mark.parametrize("V", [1000, 16385, 50000, 128256, 152064, 256000, 300007])
+# V spans one-pass clusters of 1, 3, 6, 7, 8 and 10 CTAs (the shared-memory
+# kernel's rule: ceil(V / 24576) CTAs up to 8, else up to 32768 columns each),
+# and a V past 16 CTAs of 32768 columns (and not a multiple of 8) that takes the
+# multi-pass kernels.
+@pytest.mark.parametrize("V", [1000, 16385, 50000, 128256, 152064, 256000, 300007, 600011])
 @pytest.mark.parametrize("mode", ["mean_inplace", "sum", "none_rowgrad", "loss_only"])
 def test_cross_entropy_across_cluster_sizes(V, mode):
     BT = 48
@@ -437,11 +439,13 @@ def test_cross_entropy_one_pass_edge_rows():
 
 @pytest.mark.parametrize("V", [128256, 50021, 16391, 7])
 def test_cross_entropy_one_pass_matches_multipass(monkeypatch, V):
-    """The one-pass kernels (slice staged in shared memory, the default, and slice in
-    registers, FLCE_CE=regs) agree with the oracle, with the partials + combine + grad
-    kernels, and with each other bit for bit (same arithmetic in the same order).
-    Ragged V leaves a tail of fewer than 8 columns in the last CTA's slice; rows are
-    padded to 16 bytes and the padding columns must stay untouched."""
+    """The one-pass kernels agree with the oracle and with the partials + combine +
+    grad kernels: the shared-memory kernel with its default CTA count and with
+    16384-column slices (FLCE_CE_SLICE), and the register kernel (FLCE_CE=regs). With
+    the same 16384-column slices the shared-memory and register kernels take the
+    same arithmetic in the same order, so they agree bit for bit. Ragged V leaves a
+    tail of fewer than 8 columns in the last CTA's slice; rows are padded to 16
+    bytes and the padding columns must stay untouched."""
     import ctypes
 
     from linear_cross_entropy_04_b200 import _binding as B
@@ -454,9 +458,12 @@ def test_cross_entropy_one_pass_matches_multipass(monkeypatch, V):
     assert zd.stride(0) == Vp
     gp = torch.full((256, Vp), 7.0, dtype=torch.bfloat16, device="cuda")
     out = {}
-    for mode in ("", "regs", "multipass"):
-        if mode:
-            monkeypatch.setenv("FLCE_CE", mode)
+    for mode, env in (("default", {}), ("slice16384", {"FLCE_CE_SLICE": "16384"}), ("regs", {"FLCE_CE": "regs"}),
+                      ("multipass", {"FLCE_CE": "multipass"})):
+        monkeypatch.delenv("FLCE_CE", raising=False)
+        monkeypatch.delenv("FLCE_CE_SLICE", raising=False)
+        for k, v in env.items():
+            monkeypatch.setenv(k, v)
         g = gp[:, :V]
         loss = torch.empty((), dtype=torch.float32, device="cuda")
         tz, tt, tl, tg = B.tensor(zd), B.tensor(td), B.tensor(loss), B.tensor(g)
@@ -469,12 +476,12 @@ def test_cross_entropy_one_pass_matches_multipass(monkeypatch, V):
     ref = oracle.cross_entropy(z.double().numpy(), t)
     for mode, (lv, g) in out.items():
         assert rel_err(lv, ref["loss"]) <= TOL["bf16"]["loss"], mode
-        assert_grad_close(g, ref["dz"], "bf16", f"dz ({mode or 'smem'})")
-    # the two one-pass kernels take the same arithmetic in the same order
-    assert out[""][0] == out["regs"][0] and torch.equal(out[""][1], out["regs"][1])
-    assert rel_err(out[""][0], out["multipass"][0]) <= 1e-5
-    d = (out[""][1].float() - out["multipass"][1].float()).abs().max().item()
-    assert d <= 2 ** -8 * out["multipass"][1].float().abs().max().item(), d
+        assert_grad_close(g, ref["dz"], "bf16", f"dz ({mode})")
+    assert out["slice16384"][0] == out["regs"][0] and torch.equal(out["slice16384"][1], out["regs"][1])
+    for mode in ("default", "slice16384"):
+        assert rel_err(out[mode][0], out["multipass"][0]) <= 1e-5
+        d = (out[mode][1].float() - out["multipass"][1].float()).abs().max().item()
+        assert d <= 2 ** -8 * out["multipass"][1].float().abs().max().item(), (mode, d)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
