@@ -216,35 +216,54 @@ struct DlogitsArgs {
   const float* row_grad;  // optional [rows] at chunk row 0
 };
 
+// Each thread owns DL_VECS groups of 8 columns, 2048 columns apart, and issues
+// all their loads before any store; an ignored row is written as zeros without
+// being read.
+constexpr int DL_VECS = 4;
+constexpr int DL_COLS = 256 * 8 * DL_VECS;  // columns per block
 template <typename T>
 __global__ void __launch_bounds__(256) dlogits_kernel(DlogitsArgs<T> a) {
   const int64_t r = blockIdx.y;
-  const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (c0 >= a.V) return;
+  const int64_t cb = (int64_t)blockIdx.x * DL_COLS + threadIdx.x * 8;
   const int64_t t = a.target[r];
   const bool valid = target_valid(t, a.V, a.ignore_index);
+  T* d = a.e + r * a.lde;
+  if (!valid) {
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < DL_VECS; ++u) {
+      const int64_t c0 = cb + u * 2048;
+      if (c0 + 8 <= a.V) Vec8<T>::store(d + c0, z);
+      else for (int k = 0; c0 + k < a.V && k < 8; ++k) Vec8<T>::st1(d + c0 + k, 0.f);
+    }
+    return;
+  }
   const float scale = mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f);
-  const float f = a.factor[(c0 >> a.tile_shift) * a.ldp + r];
-  const T* s = a.src + r * a.lds + c0;
-  T* d = a.e + r * a.lde + c0;
-  float v[8];
-  const bool full = c0 + 8 <= a.V;
-  if (full) {
-    Vec8<T>::load(s, v);
-  } else {
+  const T* s = a.src + r * a.lds;
+  float v[DL_VECS][8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = c0 + k < a.V ? Vec8<T>::ld1(s + k) : 0.f;
+  for (int u = 0; u < DL_VECS; ++u) {
+    const int64_t c0 = cb + u * 2048;
+    if (c0 + 8 <= a.V) {
+      Vec8<T>::load(s + c0, v[u]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[u][k] = c0 + k < a.V ? Vec8<T>::ld1(s + c0 + k) : 0.f;
+    }
   }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float x = valid ? v[k] * f : 0.f;
-    if (valid && c0 + k == t) x -= scale;
-    v[k] = x;
-  }
-  if (full) {
-    Vec8<T>::store(d, v);
-  } else {
-    for (int k = 0; k < 8 && c0 + k < a.V; ++k) Vec8<T>::st1(d + k, v[k]);
+  for (int u = 0; u < DL_VECS; ++u) {
+    const int64_t c0 = cb + u * 2048;
+    if (c0 >= a.V) break;
+    const float f = a.factor[(c0 >> a.tile_shift) * a.ldp + r];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float x = v[u][k] * f;
+      if (c0 + k == t) x -= scale;
+      v[u][k] = x;
+    }
+    if (c0 + 8 <= a.V) Vec8<T>::store(d + c0, v[u]);
+    else for (int k = 0; k < 8 && c0 + k < a.V; ++k) Vec8<T>::st1(d + c0 + k, v[u][k]);
   }
 }
 
@@ -423,11 +442,6 @@ __device__ __forceinline__ void st_cluster_f32x2(uint32_t cluster_addr, float a,
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(cluster_addr), "f"(a), "f"(b) : "memory");
 }
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 

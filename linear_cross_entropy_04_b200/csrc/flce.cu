@@ -937,7 +937,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     // A4
     {
       const int shift = dt == FLCE_BF16 ? 8 : 6;
-      const dim3 grid((unsigned)ceil_div(ceil_div(V, 8), 256), (unsigned)rows);
+      const dim3 grid((unsigned)ceil_div(V, (int64_t)DL_COLS), (unsigned)rows);
       if (dt == FLCE_BF16) {
         __nv_bfloat16* E = static_cast<__nv_bfloat16*>(estore);
         DlogitsArgs<__nv_bfloat16> a{E, pl.lde, E, pl.lde, tgt_c, ignore_index, V, pm, pl.ldp, shift, nvalid, reduction,

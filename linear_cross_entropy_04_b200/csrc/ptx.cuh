@@ -23,6 +23,14 @@ constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 constexpr float LOG2E_F = 1.4426950408889634f;
 
+// 2^x by the MUFU instruction (subnormal results flushed to zero). Its relative
+// error is far below the 2^-8 of the bf16 values and the fp32 sums it feeds.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -115,7 +115,7 @@ struct TcParams {
   // Wide tiles in one wave: pairs [0, ksync_pairs) count their arrivals at every
   // KSYNC_EVERY-th K-block in kprog[checkpoint] (zeroed before the launch), and a
   // pair waits a bounded time at a checkpoint until every pair has passed the one
-  // KSYNC_WINDOW K-blocks back, so that the dz and W panels the tiles share stay
+  // FLCE_KSYNC_WINDOW K-blocks back, so that the dz and W panels the tiles share stay
   // in L2 between their readers. 0 = off. A performance hint only: nothing
   // depends on it for correctness.
   uint32_t* kprog;
@@ -253,8 +253,8 @@ __device__ __forceinline__ void epi_logits(const TcParams& p, const TcProblem& P
     for (int j = 0; j < 32; j += 2) {
       const int col = c * 32 + j;
       const float z0 = __uint_as_float(v[j]), z1 = __uint_as_float(v[j + 1]);
-      const float e0 = col < ncols ? exp2f(fmaf(z0, LOG2E_F, -ms)) : 0.f;
-      const float e1 = col + 1 < ncols ? exp2f(fmaf(z1, LOG2E_F, -ms)) : 0.f;
+      const float e0 = col < ncols ? ex2_approx(fmaf(z0, LOG2E_F, -ms)) : 0.f;
+      const float e1 = col + 1 < ncols ? ex2_approx(fmaf(z1, LOG2E_F, -ms)) : 0.f;
       s += e0 + e1;
       if (col == tcol) ztv = z0;
       if (col + 1 == tcol) ztv = z1;

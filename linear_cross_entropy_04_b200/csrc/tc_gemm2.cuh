@@ -71,7 +71,7 @@ constexpr int T2W_SMEM_BYTES = T2W_STAGES * T2W_STAGE_BYTES + T2_OUT_BYTES + 102
 
 // Soft K-synchronisation of one-wave wide tiles (TcParams::kprog): at every
 // KSYNC_EVERY-th K-block a pair adds one to that checkpoint's counter, then waits
-// until every synchronised pair has passed the checkpoint KSYNC_WINDOW K-blocks
+// until every synchronised pair has passed the checkpoint FLCE_KSYNC_WINDOW K-blocks
 // back (at most KSYNC_CAP_NS; after a wait that runs out the pair stops
 // synchronising for the rest of the launch). One counter load per check.
 constexpr int KSYNC_EVERY = 16;
@@ -218,8 +218,8 @@ __device__ __forceinline__ void epi_logits_tma(const TcParams& p, const TcProble
     for (int j = 0; j < 32; j += 2) {
       const int col = c * 32 + j;
       const float z0 = __uint_as_float(v[j]), z1 = __uint_as_float(v[j + 1]);
-      const float e0 = col < ncols ? exp2f(fmaf(z0, LOG2E_F, -ms)) : 0.f;
-      const float e1 = col + 1 < ncols ? exp2f(fmaf(z1, LOG2E_F, -ms)) : 0.f;
+      const float e0 = col < ncols ? ex2_approx(fmaf(z0, LOG2E_F, -ms)) : 0.f;
+      const float e1 = col + 1 < ncols ? ex2_approx(fmaf(z1, LOG2E_F, -ms)) : 0.f;
       s += e0 + e1;
       if (col == tcol) ztv = z0;
       if (col + 1 == tcol) ztv = z1;
@@ -291,8 +291,8 @@ __device__ __forceinline__ void epi_dlogits_tma(const TcParams& p, const TcProbl
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
       const int col = c * 32 + j;
-      float d0 = exp2f(fmaf(__uint_as_float(v[j]), LOG2E_F, -ls)) * sg;
-      float d1 = exp2f(fmaf(__uint_as_float(v[j + 1]), LOG2E_F, -ls)) * sg;
+      float d0 = ex2_approx(fmaf(__uint_as_float(v[j]), LOG2E_F, -ls)) * sg;
+      float d1 = ex2_approx(fmaf(__uint_as_float(v[j + 1]), LOG2E_F, -ls)) * sg;
       if (col == tcol) d0 -= sg;
       if (col + 1 == tcol) d1 -= sg;
       pk[j / 2] = pack_bf16x2(d0, d1);
