@@ -520,12 +520,18 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
   float m = fmaxf(__low2float(m2), __high2float(m2));
   m = block_reduce_256(m, true, red);
   const float ms = m == -INFINITY ? 0.f : m * LOG2E_F;  // an all -inf slice sums to 0
+  // e = exp(z - m) is summed and kept, rounded to bf16, in place of z: the
+  // gradient pass then needs one multiply per element instead of a second exp
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < CER_VPT; ++i)
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      s += ex2_approx(fmaf(bf16_lo(w[i][q]), LOG2E_F, -ms)) + ex2_approx(fmaf(bf16_hi(w[i][q]), LOG2E_F, -ms));
+    for (int q = 0; q < 4; ++q) {
+      const float e0 = ex2_approx(fmaf(bf16_lo(w[i][q]), LOG2E_F, -ms));
+      const float e1 = ex2_approx(fmaf(bf16_hi(w[i][q]), LOG2E_F, -ms));
+      s += e0 + e1;
+      w[i][q] = pack_bf16x2(e0, e1);
+    }
   s = block_reduce_256(s, false, red);
   if (threadIdx.x == 0) {
     const uint32_t slot = smem_u32(&parts[rank]);
@@ -547,6 +553,7 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
   // 0 for ignored rows: every dz of such a row is exp(.) * 0 = 0
   const float scale = valid ? mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f) : 0.f;
   const float ls = lse * LOG2E_F;
+  const float f = ex2_approx(ms - ls) * scale;  // dz = e * exp(m - lse) * scale off the target
   __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
 #pragma unroll
   for (int i = 0; i < CER_VPT; ++i) {
@@ -554,9 +561,7 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
     if (c >= end) continue;
     uint32_t o[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      o[q] = pack_bf16x2(ex2_approx(fmaf(bf16_lo(w[i][q]), LOG2E_F, -ls)) * scale,
-                         ex2_approx(fmaf(bf16_hi(w[i][q]), LOG2E_F, -ls)) * scale);
+    for (int q = 0; q < 4; ++q) o[q] = pack_bf16x2(bf16_lo(w[i][q]) * f, bf16_hi(w[i][q]) * f);
     if (c + 8 <= end) {
       *reinterpret_cast<uint4*>(dr + c) = make_uint4(o[0], o[1], o[2], o[3]);
     } else {
@@ -667,13 +672,21 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
   float m = fmaxf(__low2float(m2), __high2float(m2));
   m = block_reduce_256(m, true, red);
   const float ms = m == -INFINITY ? 0.f : m * LOG2E_F;  // an all -inf slice sums to 0
+  // e = exp(z - m) is summed and written back, rounded to bf16, over z: the
+  // gradient pass then needs one multiply per element instead of a second exp
   float s = 0.f;
   for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
     const uint4 u = zs4[v];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      s += ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ms)) + ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ms));
+    for (int q = 0; q < 4; ++q) {
+      const float e0 = ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ms));
+      const float e1 = ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ms));
+      s += e0 + e1;
+      o[q] = pack_bf16x2(e0, e1);
+    }
+    zs4[v] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   s = block_reduce_256(s, false, red);
   if (threadIdx.x == 0) {
@@ -696,20 +709,20 @@ __global__ void __launch_bounds__(CER_THREADS) ce_row_smem_kernel(CeRowArgs a, u
   // 0 for ignored rows: every dz of such a row is exp(.) * 0 = 0
   const float scale = valid ? mean_scale(a.n_valid, a.reduction) * (a.row_grad ? a.row_grad[r] : 1.f) : 0.f;
   const float ls = lse * LOG2E_F;
-  const int tl = owns_t ? t - base : -1;  // the target's column within the slice
+  const float f = ex2_approx(ms - ls) * scale;  // dz = e * exp(m - lse) * scale off the target
   for (int v = threadIdx.x; v < nv_all; v += CER_THREADS) {
     const uint4 u = zs4[v];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     uint32_t o[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float d0 = ex2_approx(fmaf(bf16_lo(w[q]), LOG2E_F, -ls)) * scale;
-      float d1 = ex2_approx(fmaf(bf16_hi(w[q]), LOG2E_F, -ls)) * scale;
-      if (v * 8 + 2 * q == tl) d0 -= scale;
-      if (v * 8 + 2 * q + 1 == tl) d1 -= scale;
-      o[q] = pack_bf16x2(d0, d1);
-    }
+    for (int q = 0; q < 4; ++q) o[q] = pack_bf16x2(bf16_lo(w[q]) * f, bf16_hi(w[q]) * f);
     zs4[v] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (owns_t) {
+    // the target column, from z_t itself: exp(z_t - lse) * scale - scale
+    __syncthreads();  // the vector that holds it has been written
+    if (threadIdx.x == 0)
+      zs[t - base] = __bfloat16_as_ushort(__float2bfloat16_rn(ex2_approx(fmaf(zt, LOG2E_F, -ls)) * scale - scale));
   }
   __nv_bfloat16* dr = a.dz + (int64_t)r * a.ldd;
   fence_proxy_async_smem();  // this thread's writes, before the bulk copy reads them
