@@ -251,8 +251,9 @@ FLCE_API flce_status flce_count_valid(const flce_tensor* target, int64_t V, int6
  * a 16-CTA cluster) take one pass: a thread-block cluster per row reads the
  * logits once and writes the gradient once, with a workspace of N and the
  * per-row losses only. Each CTA of the cluster stages its slice of the row in
- * shared memory: ceil(V / 24576) CTAs up to 8, else slices of up to 32768
- * columns (FLCE_CE_SLICE=<columns> sets the slice). f32 logits and longer rows take three passes (per-tile
+ * shared memory: ceil(V / 25600) CTAs while that fits the device's largest
+ * cluster, else slices of up to 32768 columns (FLCE_CE_SLICE=<columns> sets
+ * the slice). f32 logits and longer rows take three passes (per-tile
  * partials, row combine, gradient) with a per-(row, 1024-column tile) partials
  * workspace. The workspace comes from the library's memory pool.
  */

@@ -508,21 +508,26 @@ bool ce_slice_in_registers() {
 
 // CTAs per row (the cluster size) of the shared-memory one-pass CE kernel; each
 // stages ceil(V / C) columns, rounded up to 8, in shared memory (2 bytes each, at
-// most kCeSliceMax columns). Measured on B200 (4096 rows): clusters of 6-8 CTAs
-// with 3-5 CTAs per SM run fastest (V = 128256: 0.412 ms with 6 CTAs of 21376
-// columns, against 0.450 with 8 and 0.437 with 4; V = 256000: 0.898 ms with 8 of
-// 32000, against 0.973 with 11 and 0.970 with 16). So C = ceil(V / 24576), or, when
-// that is above 8, the larger of 8 and ceil(V / 32768). FLCE_CE_SLICE=<columns>
-// (a multiple of 8 in [2048, 32768]) sets the slice instead: C = ceil(V / slice).
-int64_t ce_smem_ctas(int64_t V) {
+// most kCeSliceMax columns). What decides the speed is how many CTAs share an SM,
+// which the slice's shared memory sets (5 up to about 22500 columns, 4 up to about
+// 28000, 3 beyond), against how many CTAs meet at each row's exchange. Measured on
+// B200 (4096 rows, one exponential per element): V = 32000: 0.107 ms with 2 CTAs;
+// 50000: 0.154 with 2 (0.158 with 3); 128256: 0.374 with 6 (0.377 with 7, 0.382
+// with 5); 152064: 0.447 with 7, 0.453 with 6; 256000: 0.776 with 10 of 25600
+// columns, against 0.815 with 8 and 0.805 with 12. So C = ceil(V / 25600), or,
+// when that is above the largest cluster the device runs (max_cluster: 16 on
+// B200, else 8), ceil(V / 32768); above that the multi-pass kernels take the row.
+// FLCE_CE_SLICE=<columns> (a multiple of 8 in [2048, 32768]) sets the slice
+// instead: C = ceil(V / slice).
+int64_t ce_smem_ctas(int64_t V, int max_cluster) {
   const char* s = std::getenv("FLCE_CE_SLICE");
   if (s && *s) {
     char* end = nullptr;
     const long v = std::strtol(s, &end, 10);
     if (end != s && *end == '\0' && v >= 2048 && v <= kCeSliceMax && v % 8 == 0) return ceil_div(V, v);
   }
-  const int64_t c = ceil_div(V, 24576);
-  return c <= 8 ? c : std::max<int64_t>(8, ceil_div(V, kCeSliceMax));
+  const int64_t c = ceil_div(V, 25600);
+  return c <= max_cluster ? c : ceil_div(V, kCeSliceMax);
 }
 
 // Share of `units` workers kept busy over the waves of `tiles` equal tiles.
@@ -1167,7 +1172,7 @@ flce_status run_ce(const flce_tensor* Z, const flce_tensor* target, int64_t igno
   // bf16 rows up to (slice columns) * (largest cluster) take a one-pass cluster
   // kernel, which needs no partials; the rest take partials + combine + grad
   const bool regs = ce_slice_in_registers();
-  const int64_t cer_c64 = regs ? ceil_div(V, CER_SLICE) : ce_smem_ctas(V);
+  const int64_t cer_c64 = regs ? ceil_div(V, CER_SLICE) : ce_smem_ctas(V, dev->ce_max_cluster);
   const int cer_c = (int)std::min<int64_t>(cer_c64, 1 << 20);
   const bool one_pass = dt == FLCE_BF16 && cer_c <= dev->ce_max_cluster && ce_one_pass_enabled();
   const int64_t ntile = one_pass ? 0 : ceil_div(V, 1 << shift), ldp = round_up(BT, 32);

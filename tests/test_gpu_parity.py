@@ -375,8 +375,8 @@ def _ce_inputs(seed, BT, V, ignore_every=6):
     return z, t
 
 
-# V spans one-pass clusters of 1, 3, 6, 7, 8 and 10 CTAs (the shared-memory
-# kernel's rule: ceil(V / 24576) CTAs up to 8, else up to 32768 columns each),
+# V spans one-pass clusters of 1, 2, 6, 10 and 12 CTAs (the shared-memory
+# kernel's rule: ceil(V / 25600) CTAs up to 16, else up to 32768 columns each),
 # and a V past 16 CTAs of 32768 columns (and not a multiple of 8) that takes the
 # multi-pass kernels.
 @pytest.mark.parametrize("V", [1000, 16385, 50000, 128256, 152064, 256000, 300007, 600011])
