@@ -10,7 +10,9 @@ larger than the 126 MB L2, so no L2 flush is needed between steps.
 
 With N > 1 (torchrun), every rank runs its own batch (weak scaling) with a
 replica of W, and the step adds the data-parallel exchange: an all-reduce of
-the non-ignored row count before the loss, then of the loss and of grad_W.
+the non-ignored row count before the loss, then of the loss, then grad_W
+summed over ranks (below). --dp takes that path, collectives included, on one
+rank too.
 
 --impl reference times the float64 CPU oracle on bounded samples of the same
 workload (rank 0 only); it is the slow baseline the pages' method is exact to.
@@ -18,8 +20,11 @@ workload (rank 0 only); it is the slow baseline the pages' method is exact to.
 Other paths (one GPU, their own JSON lines):
   --path ce                 logits-given cross-entropy vs torch cross_entropy + backward
   --path preference --kind  a fused-linear preference-loss step vs PyTorch on materialised logits
---dp-fused-grad-w (N > 1) replaces the grad_W all-reduce by the reduce-scatter the
-grad_W GEMM does itself into symmetric-memory shards.
+With N > 1 grad_W is reduce-scattered by rows after the step (NCCL; each rank keeps
+V/N rows, the sharded-gradient setting of the pages' FSDP benchmark);
+--grad-w-exchange all_reduce gives every rank all of it, and --grad-w-exchange fused
+(or --dp-fused-grad-w) lets the grad_W GEMM's epilogue add each tile into the owner
+rank's symmetric-memory shard over NVLink.
 """
 from __future__ import annotations
 
@@ -58,9 +63,14 @@ def parse():
                     help="stored: row chunks keep their logits store (6*BT*H*V tensor FLOPs, the default); "
                          "recompute: vocabulary chunks, logits rebuilt after an lse pass (8*BT*H*V)")
     ap.add_argument("--workspace-limit-mib", type=int, default=0, help="chunk store budget (0: the library default)")
-    ap.add_argument("--dp-fused-grad-w", action="store_true",
-                    help="N > 1: reduce-scatter grad_W inside the grad_W GEMM over NVLink (symmetric memory) "
-                         "instead of an NCCL all-reduce after it")
+    ap.add_argument("--grad-w-exchange", default="reduce_scatter", choices=["reduce_scatter", "all_reduce", "fused"],
+                    help="N > 1: how grad_W is summed over ranks. reduce_scatter (default): NCCL reduce-scatter "
+                         "after the step, each rank keeps V/N rows (the sharded-gradient setting of the pages' "
+                         "FSDP benchmark); all_reduce: every rank gets all of grad_W; fused: the grad_W GEMM's "
+                         "epilogue adds each tile into the owner rank's shard over NVLink (symmetric memory)")
+    ap.add_argument("--dp-fused-grad-w", action="store_true", help="the same as --grad-w-exchange fused")
+    ap.add_argument("--dp", action="store_true",
+                    help="take the data-parallel code path (collectives included) even on one rank")
     ap.add_argument("--path", default="flce", choices=["flce", "ce", "preference"],
                     help="flce: the fused lm_head + loss step (default); ce: cross-entropy of given logits; "
                          "preference: a fused-linear preference loss step (--kind)")
@@ -71,6 +81,22 @@ def parse():
     ap.add_argument("--H", type=int, default=0, help="profiling: hidden size override")
     ap.add_argument("--V", type=int, default=0, help="profiling: vocabulary size override")
     return ap.parse_args()
+
+
+EXCHANGE_NAMES = {"reduce_scatter": "NCCL reduce-scatter by rows (each rank keeps V/N rows of grad_W)",
+                  "all_reduce": "NCCL all-reduce", "fused": "fused reduce-scatter in the grad_W GEMM"}
+
+
+def grad_w_exchange(args, V: int, world: int):
+    """How grad_W is summed over `world` ranks (None on one GPU, unless --dp).
+    The row reduce-scatter needs V divisible by the world size; otherwise
+    all-reduce."""
+    if world <= 1 and not args.dp:
+        return None
+    ex = "fused" if args.dp_fused_grad_w else args.grad_w_exchange
+    if ex == "reduce_scatter" and V % world:
+        return "all_reduce"
+    return ex
 
 
 def workload(args):
@@ -530,9 +556,15 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    if world > 1:
+    dp = world > 1 or args.dp  # the data-parallel code path, collectives included
+    if dp:
         import datetime
 
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29531")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     w = workload(args)
     d = make_inputs(w, seed=w.seed + rank)
@@ -550,19 +582,23 @@ def main():
 
     from linear_cross_entropy_04_b200.dp import dp_fused_linear_cross_entropy
 
+    exchange = grad_w_exchange(args, w.V, world)
+
     def step(flags=0):
-        if world > 1 and args.dp_fused_grad_w:
+        if exchange == "fused":
             # data-parallel step, grad_W reduce-scattered by the grad_W GEMM's epilogue
             dp_fused_linear_cross_entropy(X, W, t, fused_grad_W=True, flags=flags, **kw)
-        elif world > 1:
-            # data-parallel step: all-reduce N before the loss, then loss and grad_W
-            dp_fused_linear_cross_entropy(X, W, t, out=(loss, gX, gW), flags=flags, **kw)
+        elif exchange is not None:
+            # data-parallel step: all-reduce N before the loss, then the loss and grad_W
+            # (reduce-scattered by rows, or all-reduced)
+            dp_fused_linear_cross_entropy(X, W, t, out=(loss, gX, gW), shard_grad_W=exchange == "reduce_scatter",
+                                          flags=flags, **kw)
         else:
             flce.fused_linear_cross_entropy(X, W, t, out=(loss, gX, gW), flags=flags, **kw)
 
     # launch count and workspace of one step (untimed; every rank does the same)
     st = flce.fused_linear_cross_entropy(X, W, t, out=(loss, gX, gW), return_stats=True, **kw)[3]
-    launches_per_step = st["kernel_launches"] + (1 if world > 1 else 0)
+    launches_per_step = st["kernel_launches"] + (1 if dp else 0)  # the data-parallel path counts N itself
 
     mem0 = torch.cuda.memory_allocated(dev)
     torch.cuda.reset_peak_memory_stats(dev)
@@ -576,7 +612,7 @@ def main():
 
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
+    if dp:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
@@ -588,10 +624,10 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         clk.mark_end()
-    if world > 1:
+    if dp:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
-    if world > 1:
+    if dp:
         mt = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(mt, op=dist.ReduceOp.MAX)
         ms = float(mt.item())
@@ -637,7 +673,7 @@ def main():
     # back out; HostPipeline overlaps step i's upload with step i-1's compute
     # and step i-2's download on separate streams (wall clock, both ends synced)
     e2e = None
-    if world == 1 and args.e2e_steps > 0:
+    if exchange is None and args.e2e_steps > 0:
         from linear_cross_entropy_04_b200.pipeline import HostPipeline
 
         Xh = X.cpu().pin_memory()
@@ -688,6 +724,56 @@ def main():
                                     "on two streams, best of 4 (wall clock)"}
         del up, dn, Xh, Wh, th, houts
 
+    # several ranks: the data-parallel call itself, end to end, through the same
+    # host pipeline. Every step each rank copies its X, W and target in from pinned
+    # host memory, runs the step (the collectives included) and copies the loss,
+    # its grad_X and its grad_W rows back out; uploads, compute and downloads of
+    # consecutive steps overlap on three streams. CUDA events from the first
+    # upload to the last download, max over ranks.
+    if exchange in ("reduce_scatter", "all_reduce") and args.e2e_steps > 0:
+        try:
+            from linear_cross_entropy_04_b200.pipeline import HostPipeline
+
+            Xh, Wh, th = X.cpu().pin_memory(), W.cpu().pin_memory(), t.cpu().pin_memory()
+            gw_rows = w.V // world if exchange == "reduce_scatter" else w.V
+            del gX, gW
+            torch.cuda.empty_cache()
+            houts = [(torch.empty((), dtype=torch.float32).pin_memory(), torch.empty_like(Xh).pin_memory(),
+                      torch.empty((gw_rows, w.H), dtype=dt).pin_memory()) for _ in range(2)]
+
+            def dp_step(Xs, Ws, ts, out):
+                return dp_fused_linear_cross_entropy(Xs, Ws, ts, out=out, shard_grad_W=exchange == "reduce_scatter",
+                                                     **kw)
+
+            pipe = HostPipeline(w.BT, w.H, w.V, dtype=dt, slots=args.e2e_slots, step=dp_step, **kw)
+            for i in range(2):
+                pipe.submit(Xh, Wh, th, houts[i % 2])
+            pipe.synchronize()
+            torch.cuda.synchronize()
+            dist.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(pipe.s_in)
+            for i in range(args.e2e_steps):
+                pipe.submit(Xh, Wh, th, houts[i % 2])
+            e1.record(pipe.s_out)
+            pipe.synchronize()
+            torch.cuda.synchronize()
+            et = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+            ems = float(et.item())
+            h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size() + th.numel() * 8
+            d2h = 4 + houts[0][1].numel() * houts[0][1].element_size() + houts[0][2].numel() * houts[0][2].element_size()
+            e2e = {"value": w.BT * world * args.e2e_steps / (ems / 1e3), "unit": UNIT,
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems / args.e2e_steps,
+                   "slots": args.e2e_slots,
+                   "how": "per rank, the public data-parallel call (dp_fused_linear_cross_entropy) through "
+                          "HostPipeline: pinned host X, W, target copied in and loss, grad_X and this rank's "
+                          "grad_W rows copied back every step, copies overlapping compute across steps; CUDA "
+                          "events from the first upload to the last download, max over ranks; bytes are per rank"}
+            del pipe
+        except Exception as exc:  # the device-timed line above stands without it
+            e2e = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(d, args.cpu_seconds)
@@ -698,8 +784,7 @@ def main():
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded; random-init lm_head weights)",
         "config": {"workload": w.name, "BT": w.BT, "H": w.H, "V": w.V, "global_batch": w.BT * world,
                    "seq_len": w.BT, "parallelism": f"dp{world}",
-                   "grad_w_exchange": ("fused reduce-scatter in the grad_W GEMM" if args.dp_fused_grad_w
-                                       else "NCCL all-reduce") if world > 1 else None,
+                   "grad_w_exchange": EXCHANGE_NAMES.get(exchange),
                    "l2": "inputs larger than L2 (W alone is %.2f GB)" % (w.V * w.H * 2 / 1e9),
                    "chunk_rows": st["chunk_rows"], "n_chunks": st["n_chunks"],
                    "grad_w_accum": args.grad_w_accum, "schedule": args.schedule},
@@ -722,7 +807,7 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if dp:
         dist.barrier()
         dist.destroy_process_group()
     return 0

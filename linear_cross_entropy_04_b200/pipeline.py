@@ -6,11 +6,13 @@ Each step's host-to-device copies, compute and device-to-host copies run on
 three CUDA streams ordered by events, with two device slots, so step i's
 upload overlaps step i-1's compute and step i-2's download (PCIe copies in the
 two directions run concurrently). Every step still copies all of its inputs
-in and all of its results out; the compute is the library's fused call.
+in and all of its results out; the compute is the library's fused call, or
+`step` (for instance the data-parallel call, whose grad_W may come back as
+this rank's rows only).
 """
 from __future__ import annotations
 
-from typing import List, Optional, Tuple
+from typing import Callable, List, Optional, Tuple
 
 import torch
 
@@ -18,9 +20,13 @@ from .api import fused_linear_cross_entropy
 
 
 class HostPipeline:
-    def __init__(self, BT: int, H: int, V: int, dtype=torch.bfloat16, device=None, slots: int = 2, **flce_kw):
+    def __init__(self, BT: int, H: int, V: int, dtype=torch.bfloat16, device=None, slots: int = 2,
+                 step: Optional[Callable] = None, **flce_kw):
+        """step(X, W, t, out) -> (loss, grad_X, grad_W), run on the compute stream,
+        replaces the fused call; the tensors it returns are the ones copied back."""
         self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.kw = flce_kw
+        self.step = step
         self.slots = slots
         mk = lambda *s, dt=dtype: [torch.empty(*s, dtype=dt, device=self.dev) for _ in range(slots)]  # noqa: E731
         self.X, self.W, self.gX, self.gW = mk(BT, H), mk(V, H), mk(BT, H), mk(V, H)
@@ -50,14 +56,18 @@ class HostPipeline:
             self.s_run.wait_event(self.in_done[s])
             if self.used[s]:
                 self.s_run.wait_event(self.out_done[s])  # the slot's results were copied out
-            fused_linear_cross_entropy(self.X[s], self.W[s], self.t[s], out=(self.loss[s], self.gX[s], self.gW[s]),
-                                       stream=self.s_run, **self.kw)
+            out = (self.loss[s], self.gX[s], self.gW[s])
+            if self.step is None:
+                fused_linear_cross_entropy(self.X[s], self.W[s], self.t[s], out=out, stream=self.s_run, **self.kw)
+                res = out
+            else:
+                res = self.step(self.X[s], self.W[s], self.t[s], out)
             self.run_done[s].record(self.s_run)
         with torch.cuda.stream(self.s_out):
             self.s_out.wait_event(self.run_done[s])
-            out_h[0].copy_(self.loss[s], non_blocking=True)
-            out_h[1].copy_(self.gX[s], non_blocking=True)
-            out_h[2].copy_(self.gW[s], non_blocking=True)
+            for h, d in zip(out_h, res):
+                d.record_stream(self.s_out)  # a tensor the step allocated stays alive for the copy
+                h.copy_(d, non_blocking=True)
             self.out_done[s].record(self.s_out)
         self.used[s] = True
         return self.out_done[s]

@@ -98,3 +98,19 @@ def test_workload_size_overrides_rename_the_workload(bench, monkeypatch):
     assert (w.BT, w.H, w.V) == (1024, 4096, 32768) and w.name != "llama3_8b_seq"
     monkeypatch.setattr(sys, "argv", ["bench.py"])
     assert bench.workload(bench.parse()).name == "llama3_8b_seq"
+
+
+def test_grad_w_exchange_choice(bench):
+    """N > 1 reduce-scatters grad_W by rows by default (all-reduce when V does not
+    divide by N); one GPU has no exchange unless --dp asks for the path."""
+    import argparse
+
+    b = bench
+    ns = lambda **k: argparse.Namespace(**{"grad_w_exchange": "reduce_scatter", "dp_fused_grad_w": False,
+                                          "dp": False, **k})
+    assert b.grad_w_exchange(ns(), 128256, 1) is None
+    assert b.grad_w_exchange(ns(dp=True), 128256, 1) == "reduce_scatter"
+    assert b.grad_w_exchange(ns(), 128256, 8) == "reduce_scatter"
+    assert b.grad_w_exchange(ns(), 128257, 8) == "all_reduce"
+    assert b.grad_w_exchange(ns(grad_w_exchange="all_reduce"), 128256, 8) == "all_reduce"
+    assert b.grad_w_exchange(ns(dp_fused_grad_w=True), 128256, 8) == "fused"

@@ -335,6 +335,34 @@ def test_host_pipeline_matches_device_call():
         assert torch.equal(o[1], ref[1].cpu()) and torch.equal(o[2], ref[2].cpu())
 
 
+def test_host_pipeline_runs_a_caller_step():
+    """HostPipeline(step=...) runs the given step on its compute stream and copies
+    back the tensors the step returns, here a freshly allocated slice of grad_W
+    (as the data-parallel call returns this rank's rows), over several steps
+    whose slots are reused."""
+    from linear_cross_entropy_04_b200.pipeline import HostPipeline
+
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=384, H=128, V=1500)
+    X, W, t = to_dev(d)
+    ref = L().fused_linear_cross_entropy(X, W, t)
+    rows = 700
+
+    def step(Xs, Ws, ts, out):
+        lo, gx, gw = L().fused_linear_cross_entropy(Xs, Ws, ts, out=out)
+        return lo, gx, gw[:rows].clone()
+
+    Xh, Wh, th = X.cpu().pin_memory(), W.cpu().pin_memory(), t.cpu().pin_memory()
+    outs = [(torch.empty((), dtype=torch.float32).pin_memory(), torch.empty_like(Xh).pin_memory(),
+             torch.empty((rows, 128), dtype=Wh.dtype).pin_memory()) for _ in range(4)]
+    pipe = HostPipeline(384, 128, 1500, step=step)
+    for o in outs:
+        pipe.submit(Xh, Wh, th, o)
+    pipe.synchronize()
+    for o in outs:
+        assert o[0].item() == ref[0].item()
+        assert torch.equal(o[1], ref[1].cpu()) and torch.equal(o[2], ref[2][:rows].cpu())
+
+
 @pytest.mark.parametrize("every_chunk", [False, True])
 @pytest.mark.parametrize("n_shards,shard_rows,BT,chunk", [(3, 1024, 700, 256), (4, 800, 700, 256),
                                                          (4, 768, 1100, 128)])
