@@ -81,9 +81,12 @@ constexpr int T2W_SMEM_BYTES = T2W_STAGES * T2W_STAGE_BYTES + T2_OUT_BYTES + 102
 // synchronising for the rest of the launch). One counter load per check.
 constexpr int KSYNC_EVERY = 16;
 #ifndef FLCE_KSYNC_WINDOW
-#define FLCE_KSYNC_WINDOW 64
+#define FLCE_KSYNC_WINDOW 32
 #endif
-constexpr int KSYNC_LAG = FLCE_KSYNC_WINDOW / KSYNC_EVERY;  // checkpoints of lead allowed (64 K-blocks: ~50 MB)
+// checkpoints of lead allowed: 32 K-blocks keep the dz and W panels the pairs
+// share to ~25 MB (at 64 K-blocks, ~50 MB, grad_X read 1.63 GB of DRAM against
+// its 1.58 GB of operands on the same box; at 32 and 16, 1.58 GB)
+constexpr int KSYNC_LAG = FLCE_KSYNC_WINDOW / KSYNC_EVERY;
 constexpr int KSYNC_MAX_CKPT = 4096;                         // counters available (V up to 4M columns)
 constexpr uint64_t KSYNC_CAP_NS = 20000;
 
