@@ -233,12 +233,25 @@ KERNEL_SOURCES = ["linear_cross_entropy_04_b200/csrc/" + f
                   for f in ("tc_gemm2.cuh", "tc_gemm.cuh", "ptx.cuh", "aux_kernels.cuh", "flce.cu")]
 
 
+def code_only(text: str) -> str:
+    """C/C++/CUDA source with its comments removed and whitespace collapsed (no
+    string literal in these files holds a comment marker)."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
+    """sha256 (first 16 hex digits) of the code of the files that decide what the
+    GEMM launches do; comments and layout do not count."""
     import hashlib
 
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+        h.update(code_only(open(os.path.join(ROOT, f), encoding="utf-8").read()).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 

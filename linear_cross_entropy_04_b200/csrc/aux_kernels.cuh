@@ -396,11 +396,12 @@ __global__ void __launch_bounds__(256) ce_grad_kernel(CeGradArgs<T> a) {
 // A thread-block cluster of C CTAs owns one row; CTA k of the cluster holds
 // columns [k * slice, (k + 1) * slice) in registers as packed bf16 pairs
 // (CER_VPT vectors of 8 per thread, all loads issued before any use). Each CTA
-// reduces its slice to (max, sum exp(z - max)); the C pairs are exchanged
-// through distributed shared memory and one cluster barrier, after which every
-// CTA merges them in the same order into the row's lse and writes
-// dz = exp(z - lse) * scale straight from its registers, then subtracts scale
-// at the target column. The merge is the online-softmax combination of the
+// reduces its slice to (max, sum exp(z - max)), keeping e = exp(z - max) in
+// bf16 in place of z; the C pairs are exchanged through distributed shared
+// memory and one cluster barrier, after which every CTA merges them in the same
+// order into the row's lse and writes dz = e * exp(max - lse) * scale straight
+// from its registers (one exponential per element), and the target column as
+// exp(z_t - lse) * scale - scale from z_t itself. The merge is the online-softmax combination of the
 // paper review's CrossEntropy kernel with the partial tiles held on chip
 // instead of written out, so z crosses HBM once in and dz once out.
 // 64 registers per thread let 4 CTAs share an SM; exponentials use the PTX
@@ -585,9 +586,10 @@ __global__ void __launch_bounds__(CER_THREADS, FLCE_CER_MIN_BLOCKS) ce_row_clust
 // distributed shared memory), with the slice staged in shared memory instead of
 // registers: one thread moves it in with a single bulk copy (cp.async.bulk,
 // completing on an mbarrier) and the gradient goes back out with another,
-// written in place over the staged logits. The slice (<= 16384 bf16, 32 KB)
-// leaves the registers free, so 6 CTAs share an SM instead of 4, and the
-// copies are issued by the bulk-copy engine rather than 256 threads' loads.
+// written in place over the staged logits. The slice (up to 32768 bf16, 64 KB;
+// about 21-26K columns by the host's rule) leaves the registers free, so 4-5
+// CTAs share an SM instead of 4 at most, and the copies are issued by the
+// bulk-copy engine rather than 256 threads' loads.
 // Columns past the last 16-byte vector of a slice (V not a multiple of 8)
 // move with plain loads and stores.
 __device__ __forceinline__ void bulk_load_smem(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {

@@ -114,3 +114,14 @@ def test_grad_w_exchange_choice(bench):
     assert b.grad_w_exchange(ns(), 128257, 8) == "all_reduce"
     assert b.grad_w_exchange(ns(grad_w_exchange="all_reduce"), 128256, 8) == "all_reduce"
     assert b.grad_w_exchange(ns(dp_fused_grad_w=True), 128256, 8) == "fused"
+
+
+def test_source_hash_ignores_comments_but_not_code(bench):
+    """The recorded DRAM traffic stays valid across comment edits and is voided by
+    any code edit: the hash is taken over the code with comments removed."""
+    src = open(os.path.join(ROOT, "linear_cross_entropy_04_b200", "csrc", "tc_gemm2.cuh"), encoding="utf-8").read()
+    assert "constexpr int KSYNC_EVERY = 16;" in src
+    reworded = src.replace("// Soft K-synchronisation", "// Soft K-sync (reworded)").replace("/*", "/* x ")
+    assert bench.code_only(reworded) == bench.code_only(src)
+    assert bench.code_only(src.replace("KSYNC_EVERY = 16;", "KSYNC_EVERY = 8;")) != bench.code_only(src)
+    assert bench.code_only('x = 1; // a\n/* b\n c */ y =\t2;') == "x = 1; y = 2;"
