@@ -121,7 +121,7 @@ def test_source_hash_ignores_comments_but_not_code(bench):
     any code edit: the hash is taken over the code with comments removed."""
     src = open(os.path.join(ROOT, "linear_cross_entropy_04_b200", "csrc", "tc_gemm2.cuh"), encoding="utf-8").read()
     assert "constexpr int KSYNC_EVERY = 16;" in src
-    reworded = src.replace("// Soft K-synchronisation", "// Soft K-sync (reworded)").replace("/*", "/* x ")
-    assert bench.code_only(reworded) == bench.code_only(src)
+    reworded = src.replace("// Soft K-synchronisation", "// Soft K-sync (reworded)") + "\n/* a new\n block */\n"
+    assert reworded != src and bench.code_only(reworded) == bench.code_only(src)
     assert bench.code_only(src.replace("KSYNC_EVERY = 16;", "KSYNC_EVERY = 8;")) != bench.code_only(src)
     assert bench.code_only('x = 1; // a\n/* b\n c */ y =\t2;') == "x = 1; y = 2;"
