@@ -245,7 +245,9 @@ __device__ __forceinline__ void epi_logits_tma(const TcParams& p, const TcProble
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(tmE, box, (int32_t)(n0 + c * 32), (int32_t)rwarp);
+      // the store is read back only after the whole launch (525 MB later): first out of L2,
+      // ahead of the W panels that the chunk's other row tiles are about to read
+      tma_store_2d_hint(tmE, box, (int32_t)(n0 + c * 32), (int32_t)rwarp, l2_policy_evict_first());
       bulk_commit_group();
     }
     ++issued;
