@@ -81,3 +81,31 @@ def test_data_parallel_paths_on_one_rank():
     assert shape == (3000, 256) and same_w
     assert collective  # all-reduce and reduce-scatter paths equal the single-process call
     assert p.exitcode == 0
+
+
+@pytest.mark.parametrize("exchange", ["reduce_scatter", "all_reduce", "fused"])
+def test_bench_data_parallel_path_on_one_rank(exchange):
+    """`bench.py --dp` takes the multi-GPU code path (process group, collectives,
+    the chosen grad_W exchange, and, for the NCCL exchanges, the end-to-end run
+    through HostPipeline with the data-parallel call) on one rank, and prints a
+    complete line. A small workload keeps it short."""
+    import json
+    import subprocess
+    import sys
+
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()), RANK="0", WORLD_SIZE="1",
+               LOCAL_RANK="0")
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--dp", "--grad-w-exchange", exchange, "--BT", "2048",
+           "--V", "32768", "--steps", "3", "--warmup", "3", "--no-cpu-baseline", "--e2e-steps", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["n_gpus"] == 1 and line["device_error"] == 0 and line["value"] > 0
+    assert line["config"]["grad_w_exchange"].startswith(
+        {"reduce_scatter": "NCCL reduce-scatter", "all_reduce": "NCCL all-reduce", "fused": "fused"}[exchange])
+    if exchange == "fused":
+        assert line["e2e"] is None
+    else:
+        e2e = line["e2e"]
+        assert "unavailable" not in e2e and e2e["value"] > 0
+        assert e2e["h2d_bytes_per_step"] > 0 and e2e["d2h_bytes_per_step"] > 0
