@@ -46,7 +46,8 @@
 extern "C" {
 #endif
 
-#define FLCE_VERSION 110 /* 1.1.0: flce_scale_grad, flce_gemm_bf16_wait_test, FLCE_FLAG_RECOMPUTE, FLCE_FLAG_ROUTE_EVERY_CHUNK */
+#define FLCE_VERSION 120 /* 1.2.0: flce_options.grad_w_ready_event; 1.1.0: flce_scale_grad,
+                             flce_gemm_bf16_wait_test, FLCE_FLAG_RECOMPUTE, FLCE_FLAG_ROUTE_EVERY_CHUNK */
 
 #if defined(__GNUC__)
 #define FLCE_API __attribute__((visibility("default")))
@@ -165,6 +166,15 @@ typedef struct {
   int32_t n_shards;
   int64_t shard_rows;
   int64_t grad_w_shard_ld;
+  /* Optional cudaEvent_t (passed as void*), owned and created by the caller: recorded once on
+     `stream`, right after the last launch that writes grad_W (or the shards). In the stored-chunk
+     schedule the last chunk then launches its grad_W GEMM before its grad_X GEMM, so that work a
+     caller queues on another stream behind this event (a data-parallel reduction of grad_W, as
+     the pages' FSDP benchmark runs after the backward) overlaps the last grad_X GEMM, whose
+     256 x 512 tiles leave SMs free. Elsewhere it is recorded at the end of the call. Library
+     infrastructure for overlapping the data-parallel exchange; the pages define no such hook.
+     NULL = none. Added in 1.2.0. */
+  void* grad_w_ready_event;
 } flce_options;
 
 typedef struct {

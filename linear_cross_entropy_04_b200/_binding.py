@@ -41,7 +41,8 @@ class FlceOptions(ctypes.Structure):
                 ("grad_w_accum", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("n_valid", ctypes.c_void_p), ("row_loss", ctypes.c_void_p), ("lse", ctypes.c_void_p),
                 ("row_grad", ctypes.c_void_p), ("grad_w_shards", ctypes.POINTER(ctypes.c_void_p)),
-                ("n_shards", ctypes.c_int32), ("shard_rows", ctypes.c_int64), ("grad_w_shard_ld", ctypes.c_int64)]
+                ("n_shards", ctypes.c_int32), ("shard_rows", ctypes.c_int64), ("grad_w_shard_ld", ctypes.c_int64),
+                ("grad_w_ready_event", ctypes.c_void_p)]
 
 
 class FlceStats(ctypes.Structure):

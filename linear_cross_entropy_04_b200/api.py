@@ -61,7 +61,7 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
                                row_grad: Optional[torch.Tensor] = None, grad_w_shards=None,
                                shard_rows: int = 0, schedule: str = "stored",
                                flags: int = 0, stream=None, out=None, host_out=None,
-                               return_stats: bool = False):
+                               return_stats: bool = False, grad_w_ready_event=None):
     """Loss, grad_X and grad_W of cross-entropy over X W^T in one call.
 
     X [BT, H] and W [V, H] (bf16 or fp32, CUDA), target [BT] int64.
@@ -82,6 +82,10 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
     every row's logsumexp first and rebuilds the logits per vocabulary chunk
     (8*BT*H*V tensor FLOPs; the store is [BT, chunk_rows] with chunk_rows read
     as vocabulary columns, or sized from workspace_limit_bytes).
+    grad_w_ready_event (a torch.cuda.Event) is recorded on the call's stream as
+    soon as grad_W is complete: in the row-chunked schedule the last chunk runs
+    its grad_W GEMM before its grad_X GEMM, so that work queued on another stream
+    behind the event (a grad_W reduction across ranks) overlaps the grad_X GEMM.
     Returns (loss [scalar fp32], grad_X or None, grad_W or None[, stats]).
     """
     _check_reduction(reduction)
@@ -102,6 +106,10 @@ def fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torch.T
         row_grad = row_grad.to(device=X.device, dtype=torch.float32).contiguous()
     o = _options(chunk_rows, workspace_limit_bytes, grad_w_accum, flags, n_valid, row_loss, lse,
                  row_grad=row_grad)
+    if grad_w_ready_event is not None:
+        if not grad_w_ready_event.cuda_event:  # torch creates its CUDA event at the first record
+            grad_w_ready_event.record(torch.cuda.current_stream(X.device) if stream is None else stream)
+        o.grad_w_ready_event = grad_w_ready_event.cuda_event
     if grad_w_shards is not None:
         shard_ptrs = (ctypes.c_void_p * len(grad_w_shards))(*[t_.data_ptr() for t_ in grad_w_shards])
         o.grad_w_shards = ctypes.cast(shard_ptrs, ctypes.POINTER(ctypes.c_void_p))

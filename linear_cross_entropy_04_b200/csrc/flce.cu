@@ -832,6 +832,16 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
   }
   if (cudaGetLastError() != cudaSuccess) return FLCE_ERR_CUDA;
 
+  // the caller's grad_W-ready event: recorded once, mid-step when the last chunk can order
+  // grad_W before grad_X, else at the end
+  const cudaEvent_t gw_event = opt ? static_cast<cudaEvent_t>(opt->grad_w_ready_event) : nullptr;
+  bool gw_event_done = false;
+  auto record_gw_event = [&]() -> flce_status {
+    if (!gw_event || gw_event_done) return FLCE_OK;
+    gw_event_done = true;
+    return cudaEventRecord(gw_event, stream) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+  };
+
   if (BT == 0) {
     if (reduction != FLCE_NONE && cudaMemsetAsync(loss->data, 0, 4, stream) != cudaSuccess) return FLCE_ERR_CUDA;
     // shards receive additions only: nothing to add for an empty batch
@@ -839,7 +849,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
                                     H * dtype_size(dt), V, stream) != cudaSuccess)
       return FLCE_ERR_CUDA;
     if (stats) stats->workspace_bytes = 0;
-    return FLCE_OK;
+    return record_gw_event();
   }
 
   Workspace ws;
@@ -1064,10 +1074,27 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
         p2.ksync_pairs = 0;
         CUtensorMap z;
         std::memset(&z, 0, sizeof(z));
-        st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0], nullptr, nullptr, gx_wide); });
-        if (st != FLCE_OK) return st;
-        st = L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1], nullptr,
-                                      route ? &shard_maps : nullptr); });
+        auto run_gx = [&] {
+          return L.run(4, [&] { launch_tc(eg, tm[0], tm[1], z, z, p1, dev, stream, &tc[0], nullptr, nullptr,
+                                          gx_wide); });
+        };
+        auto run_gw = [&] {
+          return L.run(4, [&] { launch_tc(eg, tm[2], tm[3], z, z, p2, dev, stream, &tc[1], nullptr,
+                                          route ? &shard_maps : nullptr); });
+        };
+        if (gw_event && c == pl.n_chunks - 1) {
+          // the last chunk: grad_W first, then the event, so that the caller's work behind it
+          // overlaps the grad_X GEMM
+          st = run_gw();
+          if (st != FLCE_OK) return st;
+          st = record_gw_event();
+          if (st != FLCE_OK) return st;
+          st = run_gx();
+        } else {
+          st = run_gx();
+          if (st != FLCE_OK) return st;
+          st = run_gw();
+        }
       } else if (np == 1 && gx_wide) {
         prm.nprob = 1;
         st = L.run(4, [&] { launch_tc(eg, tm[0], tm[1], tm[2], tm[3], prm, dev, stream, &tc[0], nullptr, nullptr,
@@ -1129,7 +1156,7 @@ flce_status run_flce(const flce_tensor* X, const flce_tensor* W, const flce_tens
     if (st != FLCE_OK) return st;
   }
   if (stats) stats->kernel_launches = L.launches;
-  return FLCE_OK;
+  return record_gw_event();
 }
 
 // ------------------------------------------------------------------ CE (logits given)

@@ -105,31 +105,67 @@ def dp_fused_linear_cross_entropy(X: torch.Tensor, W: torch.Tensor, target: torc
     if fused_grad_W:
         return _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, shards, count_fn,
                                 flce_fn, **kw)
+    world = dist.get_world_size(group)
+    if want_grad_W and shard_grad_W and W.shape[0] % world:
+        raise ValueError("shard_grad_W needs V divisible by the world size")
     n_valid = None
     if reduction == "mean":
         n_valid = count_fn(target, W.shape[0], ignore_index).to(torch.int64).reshape(())
         dist.all_reduce(n_valid, group=group)
+    # On GPUs the grad_W exchange starts as soon as grad_W is complete: the library
+    # records an event there (the last chunk runs its grad_W GEMM before its grad_X
+    # GEMM), and the collective runs on a side stream behind it, overlapping the
+    # last grad_X GEMM. It is issued before the loss all-reduce, so every rank
+    # issues the two in the same order and the loss's does not hold it back.
+    overlap = (want_grad_W and flce_fn is _lib_flce and X.is_cuda and dist.get_backend(group) == "nccl"
+               and kw.get("grad_w_shards") is None)
+    ev = None
+    if overlap:
+        ev = torch.cuda.Event()
+        kw = dict(kw, grad_w_ready_event=ev)
     loss, gX, gW = flce_fn(X, W, target, ignore_index, reduction, n_valid, want_grad_X, want_grad_W, **kw)
     loss = loss.reshape(())
-    dist.all_reduce(loss, group=group)
     if want_grad_W:
-        if shard_grad_W:
-            world = dist.get_world_size(group)
-            rank = dist.get_rank(group)
-            V = gW.shape[0]
-            if V % world:
-                raise ValueError("shard_grad_W needs V divisible by the world size")
-            if dist.get_backend(group) == "gloo":
-                # gloo has no reduce_scatter of one tensor: reduce all rows, keep ours
-                dist.all_reduce(gW, group=group)
-                gW = gW[rank * (V // world):(rank + 1) * (V // world)].clone()
-            else:
-                out = torch.empty_like(gW[: V // world])
-                dist.reduce_scatter_tensor(out, gW.contiguous(), group=group)
-                gW = out
+        if overlap:
+            main = torch.cuda.current_stream(X.device) if kw.get("stream") is None else kw["stream"]
+            side = _side_stream(X.device)
+            side.wait_event(ev)
+            gW.record_stream(side)  # read by the collective on the side stream
+            with torch.cuda.stream(side):
+                gW = _exchange_grad_w(gW, shard_grad_W, group)
+            main.wait_stream(side)
+            gW.record_stream(main)
         else:
-            dist.all_reduce(gW, group=group)
+            gW = _exchange_grad_w(gW, shard_grad_W, group)
+    dist.all_reduce(loss, group=group)
     return loss, gX, gW
+
+
+_side_streams = {}
+
+
+def _side_stream(device):
+    key = str(device)
+    if key not in _side_streams:
+        _side_streams[key] = torch.cuda.Stream(device)
+    return _side_streams[key]
+
+
+def _exchange_grad_w(gW, shard_grad_W, group):
+    """grad_W summed over ranks: all of it, or (shard_grad_W) this rank's V/world rows."""
+    if not shard_grad_W:
+        dist.all_reduce(gW, group=group)
+        return gW
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    V = gW.shape[0]
+    if dist.get_backend(group) == "gloo":
+        # gloo has no reduce_scatter of one tensor: reduce all rows, keep ours
+        dist.all_reduce(gW, group=group)
+        return gW[rank * (V // world):(rank + 1) * (V // world)].clone()
+    out = torch.empty_like(gW[: V // world])
+    dist.reduce_scatter_tensor(out, gW.contiguous(), group=group)
+    return out
 
 
 def _dp_fused_grad_w(X, W, target, ignore_index, reduction, group, want_grad_X, shards, count_fn, flce_fn, **kw):

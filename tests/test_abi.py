@@ -46,7 +46,7 @@ def test_binding_signatures_cover_the_header():
 
 
 def test_version_and_status_strings(lib):
-    assert lib.flce_version() == 110
+    assert lib.flce_version() == 120
     assert lib.flce_status_string(0) == b"ok"
     assert b"unsupported device" in lib.flce_status_string(3)
     assert lib.flce_status_string(99) == b"unknown status"
@@ -399,3 +399,33 @@ def test_wait_test_hook_validates(lib, monkeypatch):
     assert lib.flce_gemm_bf16_wait_test(FAKE, FAKE, FAKE, 16, 16, 16, 16, 16, 16, -1, None) == 1
     monkeypatch.setenv("FLCE_ENGINE", "1sm")
     assert lib.flce_gemm_bf16_wait_test(FAKE, FAKE, FAKE, 256, 256, 64, 64, 64, 256, 0, None) == 1
+
+
+def test_options_struct_matches_the_header():
+    """The ctypes mirror of flce_options ends with grad_w_ready_event, as the header
+    does, and has the C struct's size (compiled with gcc from the header)."""
+    import ctypes
+    import shutil
+    import subprocess
+    import tempfile
+
+    from linear_cross_entropy_04_b200 import _binding as B
+
+    names = [f for f, _ in B.FlceOptions._fields_]
+    assert names[-1] == "grad_w_ready_event"
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "sz.c")
+        with open(src, "w") as f:
+            f.write('#include <stdio.h>\n#include <stddef.h>\n#include "flce.h"\n'
+                    'int main(void) { printf("%zu %zu\\n", sizeof(flce_options), '
+                    'offsetof(flce_options, grad_w_ready_event)); return 0; }\n')
+        exe = os.path.join(d, "sz")
+        r = subprocess.run([gcc, "-std=c99", "-I", os.path.join(ROOT, "include"), src, "-o", exe],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+        size, off = map(int, subprocess.run([exe], capture_output=True, text=True).stdout.split())
+    assert size == ctypes.sizeof(B.FlceOptions)
+    assert off == B.FlceOptions.grad_w_ready_event.offset

@@ -335,6 +335,36 @@ def test_host_pipeline_matches_device_call():
         assert torch.equal(o[1], ref[1].cpu()) and torch.equal(o[2], ref[2].cpu())
 
 
+def test_grad_w_ready_event_marks_a_complete_grad_W_before_the_end():
+    """grad_w_ready_event: the library records it as soon as grad_W is complete. A
+    copy queued on another stream behind it sees the final grad_W; the grad_X GEMM
+    of the last chunk (launched after grad_W when the event is given) still runs
+    after it; and the results equal the call without the event bit for bit. The
+    recompute schedule records it at the end."""
+    d = make_inputs(WORKLOADS["llama3_8b_seq"], BT=4096, H=4096, V=32768)
+    X, W, t = to_dev(d)
+    ref = L().fused_linear_cross_entropy(X, W, t)
+    side = torch.cuda.Stream()
+    for schedule in ("stored", "recompute"):
+        ref_s = ref if schedule == "stored" else L().fused_linear_cross_entropy(X, W, t, schedule=schedule)
+        ev = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        loss, gX, gW = L().fused_linear_cross_entropy(X, W, t, grad_w_ready_event=ev, schedule=schedule)
+        end.record()
+        side.wait_event(ev)
+        with torch.cuda.stream(side):
+            snap = gW.clone()
+        torch.cuda.synchronize()
+        assert L().device_error() == 0
+        assert torch.equal(snap, ref_s[2]) and torch.equal(gW, ref_s[2]) and torch.equal(gX, ref_s[1])
+        assert loss.item() == ref_s[0].item()
+        gap = ev.elapsed_time(end)
+        if schedule == "stored":
+            assert gap > 0.05, gap  # the last grad_X GEMM (4096 x 2048 x 32768) ran after the event
+        else:
+            assert gap >= 0.0
+
+
 def test_host_pipeline_runs_a_caller_step():
     """HostPipeline(step=...) runs the given step on its compute stream and copies
     back the tensors the step returns, here a freshly allocated slice of grad_W
