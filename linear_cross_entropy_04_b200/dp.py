@@ -7,9 +7,11 @@ exchanges, done with the process group's collectives (NCCL over NVLink on GPUs):
 
   1. all_reduce(N)      the mean denominator counts non-ignored rows of every
                         rank, and the in-place dlogits already divide by it;
-  2. all_reduce(loss)   each rank's loss is its rows' sum / N, so the sum over
-                        ranks is the global mean;
-  3. all_reduce(grad_W) (or reduce_scatter of its rows, for sharded grad_W).
+  2. all_reduce(grad_W) (or reduce_scatter of its rows, for sharded grad_W);
+                        on GPUs it starts on a side stream as soon as grad_W
+                        is complete and overlaps the step's last grad_X GEMM;
+  3. all_reduce(loss)   each rank's loss is its rows' sum / N, so the sum over
+                        ranks is the global mean.
 
 grad_X stays local. With fused_grad_W the third exchange disappears: the
 grad_W GEMM adds each output box into the owner rank's shard itself (NVLink,
