@@ -363,6 +363,18 @@ def test_grad_w_ready_event_marks_a_complete_grad_W_before_the_end():
             assert gap > 0.05, gap  # the last grad_X GEMM (4096 x 2048 x 32768) ran after the event
         else:
             assert gap >= 0.0
+    # grad_W only, and grad_X with grad_W in one launch: recorded after the last grad_W launch
+    small = make_inputs(WORKLOADS["llama3_8b_seq"], BT=700, H=256, V=3000)
+    Xs, Ws, ts = to_dev(small)
+    for kw in ({"want_grad_X": False}, {"flags": 0, "chunk_rows": 256}):
+        ref_k = L().fused_linear_cross_entropy(Xs, Ws, ts, **kw)
+        ev = torch.cuda.Event()
+        lo, gx, gw = L().fused_linear_cross_entropy(Xs, Ws, ts, grad_w_ready_event=ev, **kw)
+        side.wait_event(ev)
+        with torch.cuda.stream(side):
+            snap = gw.clone()
+        torch.cuda.synchronize()
+        assert torch.equal(snap, ref_k[2]) and torch.equal(gw, ref_k[2]), kw
 
 
 def test_host_pipeline_runs_a_caller_step():
