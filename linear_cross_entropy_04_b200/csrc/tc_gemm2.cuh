@@ -52,7 +52,16 @@ constexpr int T2_A_BYTES = T2_HALF * T2_BK * 2;  // 16 KB
 constexpr int T2_B_BYTES = T2_HALF * T2_BK * 2;  // 16 KB
 constexpr int T2_STAGE_BYTES = T2_A_BYTES + T2_B_BYTES;
 constexpr int T2_STAGE_OUT_BYTES = 32 * 32 * 2;  // one 32 x 32 bf16 staging box
-constexpr int T2_OUT_BYTES = 4 * 2 * T2_STAGE_OUT_BYTES;  // 4 epilogue warps x 2 boxes
+// Staging boxes per epilogue warp (a power of two): a box is reused once the
+// TMA store (or L2 reduce-add) issued from it FLCE_OUT_BOXES stores ago has read
+// it. Four instead of two cut the 16-chunk Llama-3-8B step by 0.5% (15 of its 16
+// grad_W launches add into grad_W in L2); the 2-chunk step did not move.
+#ifndef FLCE_OUT_BOXES
+#define FLCE_OUT_BOXES 4
+#endif
+constexpr int T2_OUT_BOXES = FLCE_OUT_BOXES;
+static_assert((T2_OUT_BOXES & (T2_OUT_BOXES - 1)) == 0, "a power of two");
+constexpr int T2_OUT_BYTES = 4 * T2_OUT_BOXES * T2_STAGE_OUT_BYTES;
 constexpr int T2_SMEM_BYTES = T2_STAGES * T2_STAGE_BYTES + T2_OUT_BYTES + 1024 + 256;
 
 // Wide tiles (256 x 512 over the pair, for long-K problems such as grad_X):
@@ -157,9 +166,9 @@ __device__ __forceinline__ void epi_bf16_tma(const CUtensorMap* tmC, bool store,
         }
       }
     }
-    uint8_t* box = boxes + (issued & 1) * T2_STAGE_OUT_BYTES;
-    if (issued >= 2) {
-      if (lane == 0) bulk_wait_group_read<1>();  // the box written two stores ago is free again
+    uint8_t* box = boxes + (issued & (T2_OUT_BOXES - 1)) * T2_STAGE_OUT_BYTES;
+    if (issued >= (uint32_t)T2_OUT_BOXES) {
+      if (lane == 0) bulk_wait_group_read<T2_OUT_BOXES - 1>();  // the box written two stores ago is free again
       __syncwarp();
     }
     uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
@@ -234,9 +243,9 @@ __device__ __forceinline__ void epi_logits_tma(const TcParams& p, const TcProble
       pk[j / 2] = pack_bf16x2(e0, e1);
     }
     if (!g.store || rwarp >= P.M || c * 32 >= ncols) continue;  // no store / box wholly outside: warp-uniform
-    uint8_t* box = boxes + (issued & 1) * T2_STAGE_OUT_BYTES;
-    if (issued >= 2) {
-      if (lane == 0) bulk_wait_group_read<1>();
+    uint8_t* box = boxes + (issued & (T2_OUT_BOXES - 1)) * T2_STAGE_OUT_BYTES;
+    if (issued >= (uint32_t)T2_OUT_BOXES) {
+      if (lane == 0) bulk_wait_group_read<T2_OUT_BOXES - 1>();
       __syncwarp();
     }
     uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
@@ -307,9 +316,9 @@ __device__ __forceinline__ void epi_dlogits_tma(const TcParams& p, const TcProbl
       if (col + 1 == tcol) d1 -= sg;
       pk[j / 2] = pack_bf16x2(d0, d1);
     }
-    uint8_t* box = boxes + (issued & 1) * T2_STAGE_OUT_BYTES;
-    if (issued >= 2) {
-      if (lane == 0) bulk_wait_group_read<1>();
+    uint8_t* box = boxes + (issued & (T2_OUT_BOXES - 1)) * T2_STAGE_OUT_BYTES;
+    if (issued >= (uint32_t)T2_OUT_BOXES) {
+      if (lane == 0) bulk_wait_group_read<T2_OUT_BOXES - 1>();
       __syncwarp();
     }
     uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
@@ -555,7 +564,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     // ---------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    uint8_t* my_boxes = out_boxes + (warp - 2) * 2 * T2_STAGE_OUT_BYTES;
+    uint8_t* my_boxes = out_boxes + (warp - 2) * T2_OUT_BOXES * T2_STAGE_OUT_BYTES;
     uint32_t issued = 0;  // TMA output boxes this warp has issued
     for (int i = 0; i < ntiles; ++i) {
       const Tile T = sched_tile(p, sched, pair, G, i);
