@@ -7,6 +7,7 @@ loss_fn(lm_head.weight, input, target) followed by loss.backward().
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 from typing import Optional
 
@@ -233,8 +234,22 @@ def cross_entropy(logits: torch.Tensor, target: torch.Tensor, ignore_index: int 
                   reduction: str = "mean", want_grad: bool = True, inplace: bool = False,
                   n_valid: Optional[torch.Tensor] = None, row_loss: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None, row_grad: Optional[torch.Tensor] = None, stream=None):
-    """Cross-entropy of given logits [BT, V]; the gradient may replace the logits in place."""
+    """Cross-entropy of given logits [BT, V]; the gradient may replace the logits in place.
+
+    The kernels read and write rows in 16-byte vectors. Logits whose rows are
+    not 16-byte aligned (a contiguous [BT, V] with V not a multiple of 8 for
+    bf16, of 4 for fp32) are staged through a copy with padded rows, and an
+    in-place gradient is copied back into them."""
     _check_reduction(reduction)
+    caller_logits = None
+    if logits.dim() == 2 and logits.shape[0] > 0 and not _rows_16b_aligned(logits):
+        caller_logits = logits if (want_grad and inplace) else None
+        per = 16 // logits.element_size()
+        V = logits.shape[1]
+        buf = torch.empty((logits.shape[0], V + (-V) % per), dtype=logits.dtype, device=logits.device)
+        with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+            buf[:, :V].copy_(logits)
+        logits = buf[:, :V]
     loss = torch.empty((logits.shape[0],) if reduction == "none" else (), dtype=torch.float32,
                        device=logits.device)
     grad = None
@@ -250,7 +265,15 @@ def cross_entropy(logits: torch.Tensor, target: torch.Tensor, ignore_index: int 
                                     ctypes.byref(tl), ctypes.byref(tg) if tg is not None else None,
                                     B.stream_handle(stream), ctypes.byref(o))
     B.check(rc, "flce_cross_entropy")
+    if caller_logits is not None:
+        with torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext():
+            caller_logits.copy_(grad)
+        grad = caller_logits
     return loss, grad
+
+
+def _rows_16b_aligned(t: torch.Tensor) -> bool:
+    return t.data_ptr() % 16 == 0 and (t.stride(0) * t.element_size()) % 16 == 0 and t.stride(-1) == 1
 
 
 def count_valid(target: torch.Tensor, V: int, ignore_index: int = -100, stream=None) -> torch.Tensor:

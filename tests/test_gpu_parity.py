@@ -487,6 +487,27 @@ def test_cross_entropy_across_cluster_sizes(V, mode):
         assert dz.data_ptr() == zd.data_ptr()
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_cross_entropy_unaligned_rows_are_staged(dtype, inplace):
+    """Contiguous logits whose rows are not 16-byte aligned (V = 50257) go through a
+    padded copy in the binding: results match the oracle, and an in-place gradient
+    lands in the caller's tensor."""
+    BT, V = 96, 50257
+    z, t = _ce_inputs(5, BT, V)
+    zt = z if dtype == "bf16" else z.float()
+    zd = zt.cuda()
+    assert (zd.stride(0) * zd.element_size()) % 16 != 0
+    loss, dz = L().cross_entropy(zd, torch.from_numpy(t).cuda(), inplace=inplace)
+    torch.cuda.synchronize()
+    assert L().device_error() == 0
+    ref = oracle.cross_entropy(zt.double().numpy(), t)
+    assert rel_err(loss.item(), ref["loss"]) <= TOL[dtype]["loss"]
+    assert_grad_close(dz, ref["dz"], dtype, "dz (unaligned rows)")
+    if inplace:
+        assert dz.data_ptr() == zd.data_ptr()
+
+
 def test_cross_entropy_one_pass_edge_rows():
     """All rows ignored (loss 0, dz 0), one row, and -inf logits (masked vocabulary)."""
     V = 50000
